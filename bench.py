@@ -1,0 +1,395 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 fused linear cross-entropy (FLCE): forward+backward
+tokens/s at V=131072 and the fraction of the dense bf16 tensor-core peak.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl own|reference]
+
+One step = one forward and one backward of the whole hot path over one batch
+of the workload `v131k_zipf` (N=16384 tokens as [2, 8192], H=4096, V=131072,
+Zipf(1.1) labels, 5% ignored, 'sum'), with inputs resident in HBM.  The inputs
+(hidden 128 MiB + weight 1 GiB bf16) are larger than the 126 MB L2, so no L2
+flush is needed between steps.  Multi-GPU runs are independent replicas (one
+problem per GPU, no collective on the data path): weak scaling.
+
+`--impl reference` times the float64 CPU oracle on a bounded token sample of
+the same workload (the pages publish no GPU implementation to run).
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import ctypes
+import datetime
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import flce_inputs as fi  # noqa: E402
+
+METRIC = "FLCE fwd+bwd tokens/s at V=131072; % of B200 dense bf16 tensor peak"
+UNIT = "tokens/s"
+WORKLOAD = "v131k_zipf"
+KIND_NAMES = ["fwd_gemm_softmax_stats", "fwd_merge_loss", "bwd_dz_gemm", "bwd_dhidden_gemm",
+              "bwd_dweight_gemm", "helper", "fp32_simt"]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["own", "reference"], default="own")
+    p.add_argument("--workload", default=WORKLOAD)
+    p.add_argument("--cpu-sample-tokens", type=int, default=256)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--e2e-steps", type=int, default=None)
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_uuid):
+        self.uuid = gpu_uuid
+        self.proc = None
+        self.tmp = None
+
+    def start(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "200"]
+            if self.uuid:
+                cmd += ["-i", self.uuid]
+            self.proc = subprocess.Popen(cmd, stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.tmp.flush()
+        self.tmp.seek(0)
+        rows = [r for r in csv.reader(io.StringIO(self.tmp.read())) if len(r) >= 9]
+        self.tmp.close()
+        os.unlink(self.tmp.name)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        top = max(sm)
+        loaded = [s for s in sm if s >= 0.5 * top] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- cpu baseline
+def oracle_step_sample(inp, w, tokens, W64):
+    """One fwd+bwd of the oracle on the first `tokens` rows; returns seconds."""
+    import oracle  # test infrastructure: the CPU baseline is the oracle itself
+    h = inp.hidden[:tokens].astype(np.float64)
+    y = inp.labels[:tokens]
+    t = time.perf_counter()
+    oracle.forward(h, W64, y, fi.IGNORE_INDEX, w.softcap, w.reduction)
+    oracle.backward(h, W64, y, fi.IGNORE_INDEX, w.softcap, w.reduction)
+    return time.perf_counter() - t
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 0) for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(inp, w, tokens):
+    W64 = inp.weight.astype(np.float64)
+    secs = oracle_step_sample(inp, w, tokens, W64)
+    return {"value": tokens / secs, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"float64 numpy oracle fwd+bwd on the first {tokens} tokens of "
+                      f"{w.name} (H={w.H}, V={w.V}), {secs:.2f} s"}
+
+
+def run_reference(args, rank):
+    """--impl reference: the oracle on the host cores, rank 0 only."""
+    if rank != 0:
+        return
+    w = fi.WORKLOADS[args.workload]
+    inp = fi.make_inputs(w)
+    W64 = inp.weight.astype(np.float64)
+    tokens = max(8, min(args.cpu_sample_tokens // 4, 64))
+    for _ in range(args.warmup):
+        oracle_step_sample(inp, w, tokens, W64)
+    secs = [oracle_step_sample(inp, w, tokens, W64) for _ in range(args.steps)]
+    total = sum(secs)
+    value = tokens * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "tokens": w.N, "hidden": w.H, "vocab": w.V,
+                   "sample_tokens_per_step": tokens, "labels": w.labels,
+                   "reduction": w.reduction},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"float64 oracle fwd+bwd on {tokens} tokens per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- own arm
+def source_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "lm_head_linear_tmem_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def dram_traffic(kind_name):
+    """Per-launch DRAM bytes from the committed ncu summary, if it matches the
+    current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("source_digest") != source_digest():
+        return None
+    ent = d.get("kernels", {}).get(kind_name)
+    return None if ent is None else ent.get("bytes_per_launch_full_size")
+
+
+def run_own(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import lm_head_linear_tmem_b200 as flce
+    from lm_head_linear_tmem_b200 import _native
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    lib = _native.load()
+    w = fi.WORKLOADS[args.workload]
+    inp = fi.make_inputs(w)
+    N, H, V = w.N, w.H, w.V
+
+    def bf16(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+
+    h_host = bf16(inp.hidden_bits).pin_memory()
+    y_host = torch.from_numpy(inp.labels).pin_memory()
+    h = h_host.to(dev)
+    W = bf16(inp.weight_bits).to(dev)
+    y = y_host.to(dev)
+    ws = flce.alloc_workspace(N, H, V, torch.bfloat16, dev)
+    lse = torch.empty(N, dtype=torch.float32, device=dev)
+    dh = torch.empty(N, H, dtype=torch.float32, device=dev)
+    dw = torch.empty(V, H, dtype=torch.float32, device=dev)
+
+    def step():
+        f = flce.forward(h, W, y, fi.IGNORE_INDEX, w.softcap, w.reduction, workspace=ws, lse=lse)
+        flce.backward(h, W, y, lse, ignore_index=fi.IGNORE_INDEX, softcap=w.softcap,
+                      reduction=w.reduction, workspace=ws, d_hidden=dh, d_weight=dw)
+        return f
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    _native.check(lib.flce_get_status(ctypes.c_void_p(ws.data_ptr()),
+                                      ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)),
+                  "warm-up status")
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        if uuid and not uuid.startswith("GPU-"):
+            uuid = "GPU-" + uuid
+    except Exception:
+        uuid = None
+
+    # ---- device-resident timing (the headline value)
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    lib.flce_profile_enable(1)
+    for k in range(len(KIND_NAMES)):  # drop records of the warm-up
+        lib.flce_profile_read(k, ctypes.byref(ctypes.c_double()), ctypes.byref(ctypes.c_int64()))
+    launches0 = lib.flce_launch_count()
+    st = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(args.steps):
+        step()
+    e1.record(st)
+    torch.cuda.synchronize()
+    launches = lib.flce_launch_count() - launches0
+    lib.flce_profile_enable(0)
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1)
+    kinds = {}
+    for k, name in enumerate(KIND_NAMES):
+        t = ctypes.c_double()
+        n = ctypes.c_int64()
+        lib.flce_profile_read(k, ctypes.byref(t), ctypes.byref(n))
+        if n.value:
+            kinds[name] = {"ms_total": t.value, "launches": n.value}
+    barrier()
+    if world > 1:
+        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    ms_step = ms / args.steps
+    value = world * N * args.steps / (ms / 1e3)
+
+    # ---- end to end through the API with host buffers
+    e2e_steps = args.e2e_steps or max(3, args.steps // 2)
+    loss_host = torch.empty((), dtype=torch.float32).pin_memory()
+    ntok_host = torch.empty((), dtype=torch.int64).pin_memory()
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(st)
+    for _ in range(e2e_steps):
+        h.copy_(h_host, non_blocking=True)
+        y.copy_(y_host, non_blocking=True)
+        f = step()
+        loss_host.copy_(f.loss, non_blocking=True)
+        ntok_host.copy_(f.num_tokens, non_blocking=True)
+    e1.record(st)
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1)
+    barrier()
+    if world > 1:
+        tt = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_e2e = float(tt.item())
+    e2e_value = world * N * e2e_steps / (ms_e2e / 1e3)
+    h2d = h_host.numel() * 2 + y_host.numel() * 8
+    d2h = 4 + 8
+
+    if rank != 0:
+        return None
+
+    peaks, peak_src = load_peaks()
+    flops_step = w.flops_per_step
+    # the dominant kernel (largest device time) and its roofline
+    credited = {"fwd_gemm_softmax_stats": 2.0 * N * H * V, "bwd_dz_gemm": 2.0 * N * H * V,
+                "bwd_dhidden_gemm": 2.0 * N * H * V, "bwd_dweight_gemm": 2.0 * N * H * V}
+    dom = max(kinds, key=lambda k: kinds[k]["ms_total"]) if kinds else None
+    roofline = None
+    if dom in credited:
+        per_launch_flops = credited[dom] * args.steps / kinds[dom]["launches"]
+        avg_ms = kinds[dom]["ms_total"] / kinds[dom]["launches"]
+        achieved = per_launch_flops / (avg_ms / 1e3) / 1e12
+        peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
+                    "unit": "TFLOP/s", "frac": achieved / peak,
+                    "peak_source": f"{peak_src} bf16_tflops_sustained",
+                    "traffic": dram_traffic(dom),
+                    "per_launch_flops": per_launch_flops, "avg_launch_ms": avg_ms}
+    tflops = flops_step / (ms_step / 1e3) / 1e12
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sust = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        cpu = cpu_baseline(inp, w, args.cpu_sample_tokens)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "tokens": N, "batch_shape": list(w.batch_shape),
+                   "hidden": H, "vocab": V, "labels": w.labels, "ignored": w.ignore_count,
+                   "softcap": w.softcap, "reduction": w.reduction,
+                   "parallelism": "replicas" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (weight 1 GiB bf16), no flush"},
+        "tensor_peak_pct": {"credited_tflops": tflops, "flops_per_step": flops_step,
+                            "frac_of_burst": tflops / burst, "frac_of_sustained": tflops / sust,
+                            "peak_source": peak_src},
+        "roofline": roofline,
+        "kernels": kinds,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return line
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_own(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

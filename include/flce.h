@@ -1,0 +1,148 @@
+/*
+ * flce.h -- C ABI of a fused linear cross-entropy (FLCE) for NVIDIA B200
+ * (sm_100a): the LM-head projection, an optional logit softcap, log-softmax
+ * cross-entropy against integer labels with ignore_index, 'sum' / 'mean'
+ * reduction with the num_tokens contract, forward and backward, without ever
+ * writing the [tokens, vocab] logits to device memory.
+ *
+ * What is computed (one row i per token, N rows, vocabulary V, hidden H):
+ *   Z    = hidden . weight^T                       (LM-head projection; weight is
+ *                                                   [vocab, hidden]: NeMo AutoModel
+ *                                                   linear_ce API, forward(lm_weight))
+ *   L    = softcap * tanh(Z / softcap), or L = Z when softcap == 0
+ *                                                  (modelscope/twinkle PR #335,
+ *                                                   "PR information" item 3; NeMo
+ *                                                   logit_softcapping=0 means off)
+ *   lse_i = log sum_v exp(L_iv)
+ *   loss_i = lse_i - L_i,y_i for rows with y_i != ignore_index, else 0
+ *                                                  (F.cross_entropy semantics:
+ *                                                   modelscope/twinkle PR #335,
+ *                                                   "Experiment results")
+ *   n     = #rows with y_i != ignore_index
+ *   'sum'  -> loss = sum_i loss_i,             num_tokens = n
+ *   'mean' -> loss = sum_i loss_i / max(n, 1), num_tokens = 0
+ *                                                  (modelscope/twinkle PR #335,
+ *                                                   item 1; the max(n, 1) clamp that
+ *                                                   makes an all-ignored batch give 0,
+ *                                                   never NaN: inclusionAI/
+ *                                                   Ling-3.1-flash discussion #7)
+ * The loss, lse and every stored intermediate are float32 (Modalities PR #464,
+ * "The problem": the stored tensors and the returned scalar must not be bf16);
+ * the loss sum is accumulated in float64.
+ *
+ * Backward (textbook derivative of the above):
+ *   g     = grad_output * grad_scale * ('mean' ? 1 / max(n, 1) : 1)
+ *   dZ_iv = g * (exp(L_iv - lse_i) - [v == y_i]) * (softcap > 0 ? 1 - (L_iv/softcap)^2 : 1),
+ *           0 on ignored rows
+ *   d_hidden = dZ . weight        [N, H] float32, overwritten
+ *   d_weight = dZ^T . hidden      [V, H] float32, overwritten
+ * grad_scale is the caller's micro-batch / token-count weighting
+ * (modelscope/twinkle PR #335, item 2: 1.0 for 'sum' per micro-batch; the
+ * trainer divides a 'sum' loss's gradient by the global non-padding token
+ * count, NeMo AutoModel forward(num_label_tokens)).
+ *
+ * Conventions shared by every call:
+ *  - All tensor arguments are DEVICE pointers on the current CUDA device,
+ *    row-major and densely packed, 16-byte aligned (torch allocations are).
+ *    hidden is [N, H], weight is [V, H], labels is int64 [N].
+ *  - dtype FLCE_BF16: hidden/weight hold bfloat16; the tensor-core path runs.
+ *    H must be a multiple of 8 (16-byte rows for the TMA engine).
+ *    dtype FLCE_FP32: hidden/weight hold float32; a CUDA-core path runs
+ *    (a correctness path for small problems, not tuned).
+ *  - stream is a cudaStream_t (NULL = legacy default stream).  Every call is
+ *    asynchronous on that stream and returns after enqueueing its kernels.
+ *  - The caller owns every buffer, including the workspace (at least
+ *    flce_workspace_bytes(...) bytes, 256-byte aligned).  The library does not
+ *    allocate device memory and keeps no per-call state.  Calls that share a
+ *    workspace must be ordered on one stream.
+ *  - Return value: argument and launch errors are reported synchronously.
+ *    Errors found by the kernels (a label outside [0, V) that is not
+ *    ignore_index, a pipeline wait that ran out of time) are recorded in a
+ *    status word inside the workspace; flce_get_status() synchronises the
+ *    stream and returns them.  Nothing aborts or traps.
+ */
+#ifndef FLCE_H
+#define FLCE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum flce_status {
+  FLCE_OK = 0,
+  FLCE_ERR_ARG = 1,          /* null pointer, bad enum, negative softcap, misaligned pointer */
+  FLCE_ERR_SHAPE = 2,        /* N < 0, V < 1, H < 8, H % 8 != 0 (bf16), sizes too large */
+  FLCE_ERR_LABEL_RANGE = 3,  /* (async) a label outside [0, V) that is not ignore_index */
+  FLCE_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
+  FLCE_ERR_UNSUPPORTED = 5,  /* device is not sm_100 */
+  FLCE_ERR_TIMEOUT = 6,      /* (async) a bounded pipeline wait inside a kernel ran out */
+  FLCE_ERR_WORKSPACE = 7     /* workspace smaller than flce_workspace_bytes() */
+} flce_status;
+
+typedef enum flce_reduction { FLCE_SUM = 0, FLCE_MEAN = 1 } flce_reduction;
+
+typedef enum flce_dtype { FLCE_BF16 = 0, FLCE_FP32 = 1 } flce_dtype;
+
+/* Bytes of workspace that flce_forward / flce_backward need for this shape.
+ * Returns 0 for invalid sizes.  Pure host computation. */
+size_t flce_workspace_bytes(int64_t N, int64_t H, int64_t V, int32_t dtype);
+
+/* Forward.
+ *   loss        device float[1]   'sum' or 'mean' loss (float32)
+ *   num_tokens  device int64[1]   n for 'sum', 0 for 'mean'
+ *   lse         device float[N]   log-sum-exp of every row (ignored rows included);
+ *                                 flce_backward reads it.
+ * ignore_index may be any int64; a row is ignored iff labels[i] == ignore_index.
+ * softcap must be >= 0 (0 = off).  The async status word is cleared first. */
+flce_status flce_forward(const void* hidden, const void* weight, const int64_t* labels,
+                         int64_t N, int64_t H, int64_t V, int64_t ignore_index, float softcap,
+                         int32_t reduction, int32_t dtype, float* loss, int64_t* num_tokens,
+                         float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward of the loss returned by flce_forward with the same arguments.
+ *   lse          device float[N]  from flce_forward
+ *   grad_output  device float[1]  upstream gradient of the loss; NULL means 1.0
+ *   grad_scale   host float       extra factor (micro-batch / token weighting)
+ *   num_valid    device int64[1]  n (the true count, also for 'mean');
+ *                                 NULL: the library counts it on the device
+ *   d_hidden     device float[N*H]  overwritten
+ *   d_weight     device float[V*H]  overwritten */
+flce_status flce_backward(const void* hidden, const void* weight, const int64_t* labels,
+                          const float* lse, int64_t N, int64_t H, int64_t V,
+                          int64_t ignore_index, float softcap, int32_t reduction, int32_t dtype,
+                          const float* grad_output, float grad_scale, const int64_t* num_valid,
+                          float* d_hidden, float* d_weight, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/* Synchronise `stream`, then return the first asynchronous error recorded in
+ * the workspace since the last flce_forward (FLCE_OK if none). */
+flce_status flce_get_status(const void* workspace, void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* flce_status_string(int32_t status);
+
+/* ABI version of this library (major * 10000 + minor * 100 + patch). */
+int32_t flce_version(void);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t flce_launch_count(void);
+
+/* Launch-time accounting, for benchmarks.  When enabled, the library records
+ * a CUDA event pair around every kernel it launches (on the call's stream).
+ * flce_profile_read synchronises those events and returns, for one kernel
+ * kind, the summed device time in milliseconds and the number of launches
+ * since the last read of that kind, then forgets them.
+ * Kinds: 0 forward GEMM+softmax stats, 1 forward merge/loss, 2 backward dZ
+ * GEMM, 3 backward dHidden GEMM, 4 backward dWeight GEMM, 5 small helper
+ * kernels, 6 fp32 CUDA-core path. */
+flce_status flce_profile_enable(int32_t enable);
+flce_status flce_profile_read(int32_t kind, double* total_ms, int64_t* launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLCE_H */

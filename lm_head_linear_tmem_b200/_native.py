@@ -1,0 +1,84 @@
+"""ctypes loader for the in-tree CUDA library `_flce.so` (C ABI: include/flce.h).
+
+Loading fails loudly: there is no CPU or PyTorch fallback for any FLCE step.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+
+c_i32 = ctypes.c_int32
+c_i64 = ctypes.c_int64
+c_u64 = ctypes.c_uint64
+c_f32 = ctypes.c_float
+c_f64 = ctypes.c_double
+c_size = ctypes.c_size_t
+c_vp = ctypes.c_void_p
+
+FLCE_OK = 0
+STATUS_NAMES = {
+    0: "FLCE_OK", 1: "FLCE_ERR_ARG", 2: "FLCE_ERR_SHAPE", 3: "FLCE_ERR_LABEL_RANGE",
+    4: "FLCE_ERR_CUDA", 5: "FLCE_ERR_UNSUPPORTED", 6: "FLCE_ERR_TIMEOUT",
+    7: "FLCE_ERR_WORKSPACE",
+}
+SUM, MEAN = 0, 1
+BF16, FP32 = 0, 1
+
+# Every symbol include/flce.h declares, with its ctypes signature.
+SIGNATURES = {
+    "flce_workspace_bytes": (c_size, [c_i64, c_i64, c_i64, c_i32]),
+    "flce_forward": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32, c_i32,
+                             c_i32, c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),
+    "flce_backward": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32,
+                              c_i32, c_i32, c_vp, c_f32, c_vp, c_vp, c_vp, c_vp, c_size,
+                              c_vp]),
+    "flce_get_status": (c_i32, [c_vp, c_vp]),
+    "flce_status_string": (ctypes.c_char_p, [c_i32]),
+    "flce_version": (c_i32, []),
+    "flce_launch_count": (c_u64, []),
+    "flce_profile_enable": (c_i32, [c_i32]),
+    "flce_profile_read": (c_i32, [c_i32, ctypes.POINTER(c_f64), ctypes.POINTER(c_i64)]),
+}
+
+_lib = None
+_lock = threading.Lock()
+
+
+class FlceError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+def library_path() -> str:
+    from . import build as _build
+    return _build.SO_PATH
+
+
+def load(build_if_missing: bool = True) -> ctypes.CDLL:
+    """Load (building first if needed) the CUDA library; raise if impossible."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        from . import build as _build
+        path = library_path()
+        if build_if_missing and _build.needs_build():
+            _build.build()
+        if not os.path.exists(path):
+            raise RuntimeError(f"FLCE CUDA library not found at {path}; run "
+                               "`python -m lm_head_linear_tmem_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+        return lib
+
+
+def check(status: int, where: str) -> None:
+    if status != FLCE_OK:
+        raise FlceError(status, where)

@@ -1,0 +1,324 @@
+// CUDA-core kernels of the fused linear cross-entropy: merging the forward's
+// per-vocab-tile softmax statistics into lse, the per-row loss with a
+// deterministic float64 reduction, the valid-row count, and the fp32 path
+// (plain FFMA kernels for float32 inputs; a correctness path, not tuned).
+#pragma once
+
+#include <math_constants.h>
+
+#include "tc_gemm.cuh"
+
+namespace flce {
+
+constexpr int kMergeRows = 32;
+constexpr int kMergeSplit = 8;
+constexpr int kLossThreads = 256;
+constexpr int kFinalThreads = 1024;
+
+// Merge (m, s) pairs of the log2-domain online softmax: returns the pair for
+// the union of both column sets.  (-inf, 0) is the empty set.
+__device__ __forceinline__ void merge_ms(float& M, float& S, float m, float s) {
+  if (m == -CUDART_INF_F) return;
+  if (m > M) {
+    S = (M == -CUDART_INF_F) ? s : S * exp2f(M - m) + s;
+    M = m;
+  } else {
+    S += s * exp2f(m - M);
+  }
+}
+
+// lse[row] = ln 2 * (M + log2 S) over all vocab tiles of the row.
+// Block (32 rows, 8 splits); grid ceil(N / 32).
+__global__ void __launch_bounds__(kMergeRows * kMergeSplit)
+    fwd_merge_kernel(const float* __restrict__ part_m, const float* __restrict__ part_s,
+                     int n_vt, int N, float* __restrict__ lse) {
+  __shared__ float sm[kMergeSplit][kMergeRows];
+  __shared__ float ss[kMergeSplit][kMergeRows];
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  const int row = blockIdx.x * kMergeRows + tx;
+  float M = -CUDART_INF_F, S = 0.f;
+  if (row < N) {
+    for (int vt = ty; vt < n_vt; vt += kMergeSplit) {
+      const size_t idx = static_cast<size_t>(vt) * N + row;
+      merge_ms(M, S, part_m[idx], part_s[idx]);
+    }
+  }
+  sm[ty][tx] = M;
+  ss[ty][tx] = S;
+  __syncthreads();
+  if (ty == 0 && row < N) {
+    float Mt = -CUDART_INF_F, St = 0.f;
+    for (int k = 0; k < kMergeSplit; ++k) merge_ms(Mt, St, sm[k][tx], ss[k][tx]);
+    lse[row] = (Mt + log2f(St)) * kLn2;
+  }
+}
+
+// Per-row loss lse_i - L[i, y_i] for non-ignored rows, summed in float64 per
+// block in a fixed order; rows with a label outside [0, V) that is not
+// ignore_index set the label-range status bit and contribute nothing.
+__global__ void __launch_bounds__(kLossThreads)
+    row_loss_kernel(const float* __restrict__ lse, const float* __restrict__ label_logit,
+                    const int64_t* __restrict__ labels, int N, int64_t ignore_index, int64_t V,
+                    double* __restrict__ block_loss, long long* __restrict__ block_cnt,
+                    unsigned int* status) {
+  __shared__ double sl[kLossThreads];
+  __shared__ long long sc[kLossThreads];
+  const int t = threadIdx.x;
+  const int row = blockIdx.x * kLossThreads + t;
+  double l = 0.0;
+  long long c = 0;
+  if (row < N) {
+    const int64_t y = labels[row];
+    if (y != ignore_index) {
+      if (y < 0 || y >= V) {
+        atomicOr(status, kStatusLabelRange);
+      } else {
+        l = static_cast<double>(lse[row]) - static_cast<double>(label_logit[row]);
+        c = 1;
+      }
+    }
+  }
+  sl[t] = l;
+  sc[t] = c;
+  __syncthreads();
+  for (int w = kLossThreads / 2; w > 0; w >>= 1) {
+    if (t < w) {
+      sl[t] += sl[t + w];
+      sc[t] += sc[t + w];
+    }
+    __syncthreads();
+  }
+  if (t == 0) {
+    block_loss[blockIdx.x] = sl[0];
+    block_cnt[blockIdx.x] = sc[0];
+  }
+}
+
+// One block: fixed-order float64 sum of the block partials, then the
+// reduction contract: 'sum' -> (sum, n); 'mean' -> (sum / max(n,1), 0).
+__global__ void __launch_bounds__(kFinalThreads)
+    finalize_kernel(const double* __restrict__ block_loss, const long long* __restrict__ block_cnt,
+                    int nblk, int mean, float* loss, int64_t* num_tokens, long long* n_valid_out) {
+  __shared__ double sl[kFinalThreads];
+  __shared__ long long sc[kFinalThreads];
+  const int t = threadIdx.x;
+  double l = 0.0;
+  long long c = 0;
+  for (int b = t; b < nblk; b += kFinalThreads) {
+    l += block_loss[b];
+    c += block_cnt[b];
+  }
+  sl[t] = l;
+  sc[t] = c;
+  __syncthreads();
+  for (int w = kFinalThreads / 2; w > 0; w >>= 1) {
+    if (t < w) {
+      sl[t] += sl[t + w];
+      sc[t] += sc[t + w];
+    }
+    __syncthreads();
+  }
+  if (t == 0) {
+    const long long n = sc[0];
+    const double total = sl[0];
+    if (mean) {
+      loss[0] = static_cast<float>(total / static_cast<double>(n > 0 ? n : 1));
+      num_tokens[0] = 0;
+    } else {
+      loss[0] = static_cast<float>(total);
+      num_tokens[0] = n;
+    }
+    if (n_valid_out != nullptr) *n_valid_out = n;
+  }
+}
+
+// n = #rows with label != ignore_index (one block).
+__global__ void __launch_bounds__(kFinalThreads)
+    count_valid_kernel(const int64_t* __restrict__ labels, int N, int64_t ignore_index,
+                       long long* n_valid_out) {
+  __shared__ long long sc[kFinalThreads];
+  const int t = threadIdx.x;
+  long long c = 0;
+  for (int i = t; i < N; i += kFinalThreads) c += (labels[i] != ignore_index) ? 1 : 0;
+  sc[t] = c;
+  __syncthreads();
+  for (int w = kFinalThreads / 2; w > 0; w >>= 1) {
+    if (t < w) sc[t] += sc[t + w];
+    __syncthreads();
+  }
+  if (t == 0) *n_valid_out = sc[0];
+}
+
+// ------------------------------------------------------------------ fp32 path
+constexpr int kSimtThreads = 256;
+constexpr int kSimtChunk = 1024;
+
+__device__ __forceinline__ float capped(float z, float softcap) {
+  return softcap > 0.f ? softcap * tanhf(z / softcap) : z;
+}
+
+// One block per token row: lse and the label logit, natural-log domain.
+// Dynamic smem: H floats (the row of hidden).
+__global__ void __launch_bounds__(kSimtThreads)
+    simt_fwd_kernel(const float* __restrict__ hidden, const float* __restrict__ weight,
+                    const int64_t* __restrict__ labels, int N, int H, int V, float softcap,
+                    float* __restrict__ lse, float* __restrict__ label_logit) {
+  extern __shared__ float sh[];
+  __shared__ float red_m[kSimtThreads], red_s[kSimtThreads];
+  const int row = blockIdx.x;
+  const int t = threadIdx.x;
+  for (int k = t; k < H; k += kSimtThreads) sh[k] = hidden[static_cast<size_t>(row) * H + k];
+  __syncthreads();
+  const int64_t y = labels[row];
+  float m = -CUDART_INF_F, s = 0.f;
+  for (int v = t; v < V; v += kSimtThreads) {
+    const float* w = weight + static_cast<size_t>(v) * H;
+    float z = 0.f;
+    for (int k = 0; k < H; ++k) z = fmaf(sh[k], w[k], z);
+    const float L = capped(z, softcap);
+    if (v == y) label_logit[row] = L;
+    if (L > m) {
+      s = (m == -CUDART_INF_F) ? 1.f : s * expf(m - L) + 1.f;
+      m = L;
+    } else {
+      s += expf(L - m);
+    }
+  }
+  red_m[t] = m;
+  red_s[t] = s;
+  __syncthreads();
+  for (int w = kSimtThreads / 2; w > 0; w >>= 1) {
+    if (t < w) {
+      float M = red_m[t], S = red_s[t];
+      const float m2 = red_m[t + w], s2 = red_s[t + w];
+      if (m2 != -CUDART_INF_F) {
+        if (m2 > M) {
+          S = (M == -CUDART_INF_F) ? s2 : S * expf(M - m2) + s2;
+          M = m2;
+        } else {
+          S += s2 * expf(m2 - M);
+        }
+      }
+      red_m[t] = M;
+      red_s[t] = S;
+    }
+    __syncthreads();
+  }
+  if (t == 0) lse[row] = red_m[0] + logf(red_s[0]);
+}
+
+__device__ __forceinline__ float simt_grad_scale(const float* grad_output, float grad_scale,
+                                                 const long long* n_valid, int mean) {
+  float g = (grad_output != nullptr ? grad_output[0] : 1.0f) * grad_scale;
+  if (mean) {
+    const long long n = *n_valid;
+    g /= static_cast<float>(n > 0 ? n : 1);
+  }
+  return g;
+}
+
+// One block per token row: dHidden[row] = sum_v dZ[row, v] W[v].
+// Dynamic smem: 2*H + kSimtChunk floats.
+__global__ void __launch_bounds__(kSimtThreads)
+    simt_dh_kernel(const float* __restrict__ hidden, const float* __restrict__ weight,
+                   const int64_t* __restrict__ labels, const float* __restrict__ lse, int N,
+                   int H, int V, int64_t ignore_index, float softcap, const float* grad_output,
+                   float grad_scale, const long long* n_valid, int mean,
+                   float* __restrict__ d_hidden) {
+  extern __shared__ float sh[];
+  float* h = sh;
+  float* acc = sh + H;
+  float* G = sh + 2 * H;
+  const int row = blockIdx.x;
+  const int t = threadIdx.x;
+  const int64_t y = labels[row];
+  const bool valid = (y != ignore_index);
+  const float g = simt_grad_scale(grad_output, grad_scale, n_valid, mean);
+  const float l = lse[row];
+  for (int k = t; k < H; k += kSimtThreads) {
+    h[k] = hidden[static_cast<size_t>(row) * H + k];
+    acc[k] = 0.f;
+  }
+  __syncthreads();
+  for (int v0 = 0; v0 < V; v0 += kSimtChunk) {
+    const int nv = min(kSimtChunk, V - v0);
+    for (int j = t; j < nv; j += kSimtThreads) {
+      const int v = v0 + j;
+      float gz = 0.f;
+      if (valid) {
+        const float* w = weight + static_cast<size_t>(v) * H;
+        float z = 0.f;
+        for (int k = 0; k < H; ++k) z = fmaf(h[k], w[k], z);
+        const float L = capped(z, softcap);
+        float d = expf(L - l) - (v == y ? 1.f : 0.f);
+        if (softcap > 0.f) {
+          const float u = L / softcap;
+          d *= 1.f - u * u;
+        }
+        gz = g * d;
+      }
+      G[j] = gz;
+    }
+    __syncthreads();
+    for (int k = t; k < H; k += kSimtThreads) {
+      float a = acc[k];
+      for (int j = 0; j < nv; ++j) a = fmaf(G[j], weight[static_cast<size_t>(v0 + j) * H + k], a);
+      acc[k] = a;
+    }
+    __syncthreads();
+  }
+  for (int k = t; k < H; k += kSimtThreads) d_hidden[static_cast<size_t>(row) * H + k] = acc[k];
+}
+
+// One block per vocab row: dWeight[v] = sum_i dZ[i, v] hidden[i].
+// Dynamic smem: 2*H + kSimtThreads floats.
+__global__ void __launch_bounds__(kSimtThreads)
+    simt_dw_kernel(const float* __restrict__ hidden, const float* __restrict__ weight,
+                   const int64_t* __restrict__ labels, const float* __restrict__ lse, int N,
+                   int H, int V, int64_t ignore_index, float softcap, const float* grad_output,
+                   float grad_scale, const long long* n_valid, int mean,
+                   float* __restrict__ d_weight) {
+  extern __shared__ float sh[];
+  float* w = sh;
+  float* acc = sh + H;
+  float* G = sh + 2 * H;
+  const int v = blockIdx.x;
+  const int t = threadIdx.x;
+  const float g = simt_grad_scale(grad_output, grad_scale, n_valid, mean);
+  for (int k = t; k < H; k += kSimtThreads) {
+    w[k] = weight[static_cast<size_t>(v) * H + k];
+    acc[k] = 0.f;
+  }
+  __syncthreads();
+  for (int i0 = 0; i0 < N; i0 += kSimtThreads) {
+    const int ni = min(kSimtThreads, N - i0);
+    if (t < ni) {
+      const int i = i0 + t;
+      const int64_t y = labels[i];
+      float gz = 0.f;
+      if (y != ignore_index) {
+        const float* hi = hidden + static_cast<size_t>(i) * H;
+        float z = 0.f;
+        for (int k = 0; k < H; ++k) z = fmaf(hi[k], w[k], z);
+        const float L = capped(z, softcap);
+        float d = expf(L - lse[i]) - (v == y ? 1.f : 0.f);
+        if (softcap > 0.f) {
+          const float u = L / softcap;
+          d *= 1.f - u * u;
+        }
+        gz = g * d;
+      }
+      G[t] = gz;
+    }
+    __syncthreads();
+    for (int k = t; k < H; k += kSimtThreads) {
+      float a = acc[k];
+      for (int j = 0; j < ni; ++j) a = fmaf(G[j], hidden[static_cast<size_t>(i0 + j) * H + k], a);
+      acc[k] = a;
+    }
+    __syncthreads();
+  }
+  for (int k = t; k < H; k += kSimtThreads) d_weight[static_cast<size_t>(v) * H + k] = acc[k];
+}
+
+}  // namespace flce

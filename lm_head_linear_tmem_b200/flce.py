@@ -1,0 +1,193 @@
+"""PyTorch binding of the FLCE C ABI (argument marshalling only).
+
+Every arithmetic step of the fused linear cross-entropy runs in the CUDA
+library `_flce.so`; this module only checks tensor arguments, allocates the
+outputs and the workspace with torch, and passes raw device pointers and the
+current CUDA stream.  There is no CPU or PyTorch fallback.
+
+API (names follow the pages):
+  forward(hidden, weight, labels, ignore_index=-100, softcap=0.0, reduction='sum')
+      -> FlceForward(loss, num_tokens, lse)
+  backward(hidden, weight, labels, lse, grad_output=None, grad_scale=1.0, ...)
+      -> (d_hidden, d_weight)
+  FusedLinearCrossEntropy(ignore_index=-100, logit_softcapping=0, reduction='sum')
+      an nn.Module whose forward(hidden_states, labels, lm_weight) returns the
+      loss and records `num_tokens` ('sum': non-ignored count, 'mean': 0), as
+      the NeMo AutoModel linear_ce API and modelscope/twinkle PR #335 specify.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import NamedTuple, Optional, Tuple
+
+import torch
+
+from . import _native
+
+_DTYPES = {torch.bfloat16: _native.BF16, torch.float32: _native.FP32}
+_REDUCTIONS = {"sum": _native.SUM, "mean": _native.MEAN}
+
+
+class FlceForward(NamedTuple):
+    loss: torch.Tensor        # float32 scalar
+    num_tokens: torch.Tensor  # int64 scalar ('sum': n, 'mean': 0)
+    lse: torch.Tensor         # float32 [N]
+
+
+def _lib():
+    return _native.load()
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _prep(hidden: torch.Tensor, weight: torch.Tensor, labels: torch.Tensor):
+    if not (hidden.is_cuda and weight.is_cuda and labels.is_cuda):
+        raise ValueError("hidden, weight and labels must be CUDA tensors")
+    if hidden.device != weight.device or hidden.device != labels.device:
+        raise ValueError("hidden, weight and labels must be on one device")
+    if hidden.dtype not in _DTYPES or weight.dtype != hidden.dtype:
+        raise TypeError("hidden and weight must both be bfloat16 or both float32")
+    if weight.dim() != 2:
+        raise ValueError("weight must be [vocab, hidden]")
+    H = weight.shape[1]
+    if hidden.shape[-1] != H:
+        raise ValueError("hidden's last dim must equal weight.shape[1]")
+    h2 = hidden.reshape(-1, H).contiguous()
+    y = labels.reshape(-1)
+    if y.dtype != torch.int64:
+        y = y.to(torch.int64)
+    y = y.contiguous()
+    if y.shape[0] != h2.shape[0]:
+        raise ValueError("labels must have one entry per token")
+    return h2, weight.contiguous(), y
+
+
+def workspace_bytes(N: int, H: int, V: int, dtype: torch.dtype = torch.bfloat16) -> int:
+    return int(_lib().flce_workspace_bytes(N, H, V, _DTYPES[dtype]))
+
+
+def alloc_workspace(N: int, H: int, V: int, dtype: torch.dtype, device) -> torch.Tensor:
+    n = workspace_bytes(N, H, V, dtype)
+    if n == 0:
+        raise ValueError("invalid FLCE sizes")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def status(workspace: torch.Tensor) -> int:
+    """Synchronise and return the asynchronous status recorded in `workspace`."""
+    return int(_lib().flce_get_status(ctypes.c_void_p(workspace.data_ptr()),
+                                      ctypes.c_void_p(_stream(workspace.device))))
+
+
+def forward(hidden: torch.Tensor, weight: torch.Tensor, labels: torch.Tensor,
+            ignore_index: int = -100, softcap: float = 0.0, reduction: str = "sum",
+            workspace: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+            check_status: bool = False) -> FlceForward:
+    h2, w, y = _prep(hidden, weight, labels)
+    N, H = h2.shape
+    V = w.shape[0]
+    dev = h2.device
+    if workspace is None:
+        workspace = alloc_workspace(N, H, V, h2.dtype, dev)
+    loss = torch.empty((), dtype=torch.float32, device=dev)
+    ntok = torch.empty((), dtype=torch.int64, device=dev)
+    if lse is None:
+        lse = torch.empty(N, dtype=torch.float32, device=dev)
+    st = _lib().flce_forward(_ptr(h2), _ptr(w), _ptr(y), N, H, V, int(ignore_index),
+                             float(softcap), _REDUCTIONS[reduction], _DTYPES[h2.dtype],
+                             _ptr(loss), _ptr(ntok), _ptr(lse), _ptr(workspace),
+                             workspace.numel(), _stream(dev))
+    _native.check(st, "flce_forward")
+    if check_status:
+        _native.check(status(workspace), "flce_forward (device status)")
+    return FlceForward(loss, ntok, lse)
+
+
+def backward(hidden: torch.Tensor, weight: torch.Tensor, labels: torch.Tensor,
+             lse: torch.Tensor, grad_output: Optional[torch.Tensor] = None,
+             grad_scale: float = 1.0, num_valid: Optional[torch.Tensor] = None,
+             ignore_index: int = -100, softcap: float = 0.0, reduction: str = "sum",
+             workspace: Optional[torch.Tensor] = None,
+             d_hidden: Optional[torch.Tensor] = None, d_weight: Optional[torch.Tensor] = None,
+             check_status: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+    h2, w, y = _prep(hidden, weight, labels)
+    N, H = h2.shape
+    V = w.shape[0]
+    dev = h2.device
+    if workspace is None:
+        workspace = alloc_workspace(N, H, V, h2.dtype, dev)
+    if d_hidden is None:
+        d_hidden = torch.empty((N, H), dtype=torch.float32, device=dev)
+    if d_weight is None:
+        d_weight = torch.empty((V, H), dtype=torch.float32, device=dev)
+    if grad_output is not None:
+        grad_output = grad_output.reshape(()).to(device=dev, dtype=torch.float32).contiguous()
+    if num_valid is not None:
+        num_valid = num_valid.reshape(()).to(device=dev, dtype=torch.int64).contiguous()
+    lse = lse.contiguous()
+    st = _lib().flce_backward(_ptr(h2), _ptr(w), _ptr(y), _ptr(lse), N, H, V, int(ignore_index),
+                              float(softcap), _REDUCTIONS[reduction], _DTYPES[h2.dtype],
+                              _ptr(grad_output), float(grad_scale), _ptr(num_valid),
+                              _ptr(d_hidden), _ptr(d_weight), _ptr(workspace),
+                              workspace.numel(), _stream(dev))
+    _native.check(st, "flce_backward")
+    if check_status:
+        _native.check(status(workspace), "flce_backward (device status)")
+    return d_hidden, d_weight
+
+
+class _FlceFunction(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, hidden, weight, labels, ignore_index, softcap, reduction, grad_scale):
+        out = forward(hidden, weight, labels, ignore_index, softcap, reduction)
+        ctx.save_for_backward(hidden, weight, labels, out.lse)
+        ctx.cfg = (ignore_index, softcap, reduction, grad_scale, hidden.shape)
+        ctx.mark_non_differentiable(out.num_tokens)
+        return out.loss, out.num_tokens
+
+    @staticmethod
+    def backward(ctx, grad_loss, _grad_ntok):
+        hidden, weight, labels, lse = ctx.saved_tensors
+        ignore_index, softcap, reduction, grad_scale, hshape = ctx.cfg
+        dh, dw = backward(hidden, weight, labels, lse, grad_output=grad_loss,
+                          grad_scale=grad_scale, ignore_index=ignore_index, softcap=softcap,
+                          reduction=reduction)
+        return dh.reshape(hshape), dw, None, None, None, None, None
+
+
+def fused_linear_cross_entropy(hidden, weight, labels, ignore_index: int = -100,
+                               softcap: float = 0.0, reduction: str = "sum",
+                               grad_scale: float = 1.0):
+    """Differentiable (loss, num_tokens); gradients flow to hidden and weight."""
+    return _FlceFunction.apply(hidden, weight, labels, ignore_index, softcap, reduction,
+                               grad_scale)
+
+
+class FusedLinearCrossEntropy(torch.nn.Module):
+    """Loss module with the constructor of the NeMo AutoModel linear_ce API."""
+
+    def __init__(self, ignore_index: int = -100, logit_softcapping: float = 0,
+                 reduction: str = "sum"):
+        super().__init__()
+        if reduction not in _REDUCTIONS:
+            raise ValueError("reduction must be 'sum' or 'mean'")
+        if logit_softcapping < 0:
+            raise ValueError("logit_softcapping must be >= 0")
+        self.ignore_index = ignore_index
+        self.logit_softcapping = float(logit_softcapping)
+        self.reduction = reduction
+        self.num_tokens: Optional[torch.Tensor] = None
+
+    def forward(self, hidden_states: torch.Tensor, labels: torch.Tensor,
+                lm_weight: torch.Tensor, grad_scale: float = 1.0) -> torch.Tensor:
+        loss, ntok = fused_linear_cross_entropy(hidden_states, lm_weight, labels,
+                                                self.ignore_index, self.logit_softcapping,
+                                                self.reduction, grad_scale)
+        self.num_tokens = ntok
+        return loss

@@ -1,0 +1,55 @@
+"""Helpers shared by the GPU parity tests (inputs to device, comparisons).
+
+Tolerances come from the contract of this FLCE build:
+  num_tokens, ignored-row zeros   bit-exact
+  loss                            1e-5 relative
+  dHidden, dWeight                2e-3 relative L2
+  lse (per row)                   1e-4 absolute: the row's logsumexp is an
+                                  fp32 quantity of magnitude <= ~15 here, its
+                                  fp32 grid is ~1e-6 and the tensor-core dot
+                                  products of K <= 4096 bf16 pairs carry
+                                  ~1e-6 of accumulated rounding; 1e-4 leaves a
+                                  wide margin while still catching any
+                                  dropped tile or wrong column (>= 1e-2).
+"""
+import numpy as np
+import torch
+
+import flce_inputs as fi
+
+LOSS_RTOL = 1e-5
+GRAD_RL2 = 2e-3
+LSE_ATOL = 1e-4
+
+
+def bf16_tensor(bits: np.ndarray, device="cuda") -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def f32_tensor(a: np.ndarray, device="cuda") -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+
+
+def labels_tensor(y: np.ndarray, device="cuda") -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(y, dtype=np.int64)).to(device)
+
+
+def rel_l2(got: np.ndarray, ref: np.ndarray) -> float:
+    den = float(np.linalg.norm(ref))
+    num = float(np.linalg.norm(np.asarray(got, np.float64) - ref))
+    if den == 0.0:
+        return num
+    return num / den
+
+
+def check_loss(got: float, ref: float):
+    if ref == 0.0:
+        assert got == 0.0, got
+    else:
+        assert abs(got - ref) <= LOSS_RTOL * abs(ref), (got, ref, abs(got - ref) / abs(ref))
+
+
+def small_inputs(N, H, V, seed, n_ign, w_std=0.05):
+    """Seeded ad-hoc problem with the workload recipe (bf16-quantised)."""
+    w = fi.custom_workload(N, H, V, seed=seed, w_std=w_std, ignore_count=n_ign)
+    return fi.make_inputs(w, keep_raw=True)

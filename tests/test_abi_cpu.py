@@ -1,0 +1,101 @@
+"""The C-ABI library builds, loads and exports every symbol include/flce.h
+declares; host-side argument checks answer without touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from lm_head_linear_tmem_b200 import _native, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "flce.h")
+
+FAKE = 0x10000  # a 256-aligned, never-dereferenced address for argument-check tests
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(flce_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _native.load()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("flce_forward", "flce_backward", "flce_workspace_bytes", "flce_get_status"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in _native.SIGNATURES, name
+
+
+def test_version_and_strings(lib):
+    assert lib.flce_version() >= 100
+    for code, name in _native.STATUS_NAMES.items():
+        assert lib.flce_status_string(code).decode() == name
+    assert lib.flce_status_string(99).decode() == "FLCE_ERR_UNKNOWN"
+
+
+def test_workspace_bytes(lib):
+    ws = lib.flce_workspace_bytes
+    assert ws(-1, 64, 512, 0) == 0
+    assert ws(64, 4, 512, 0) == 0
+    assert ws(64, 64, 0, 0) == 0
+    assert ws(64, 64, 512, 7) == 0
+    tiny = ws(64, 64, 512, 0)
+    assert tiny > 0 and tiny % 256 == 0
+    big = ws(16384, 4096, 131072, 0)
+    # forward partials: 512 vocab tiles x 16384 rows x (m, s) fp32 = 64 MiB;
+    # backward dZ block: 4096 x 8192 bf16 = 64 MiB
+    assert 64 * 2 ** 20 <= big < 66 * 2 ** 20
+    assert ws(0, 64, 512, 0) > 0
+    assert ws(64, 64, 512, 1) > 0
+
+
+def _fwd(lib, N=64, H=64, V=512, softcap=0.0, reduction=0, dtype=0, ws_size=None,
+         hidden=FAKE, weight=FAKE, labels=FAKE, loss=FAKE, ntok=FAKE, lse=FAKE):
+    if ws_size is None:
+        ws_size = lib.flce_workspace_bytes(N, H, V, dtype) or 1 << 20
+    return lib.flce_forward(hidden, weight, labels, N, H, V, -100, softcap, reduction, dtype,
+                            loss, ntok, lse, FAKE, ws_size, None)
+
+
+def test_argument_errors_are_synchronous(lib):
+    ARG, SHAPE, WS = 1, 2, 7
+    assert _fwd(lib, reduction=5) == ARG
+    assert _fwd(lib, dtype=3) == ARG
+    assert _fwd(lib, softcap=-1.0) == ARG
+    assert _fwd(lib, softcap=float("nan")) == ARG
+    assert _fwd(lib, softcap=float("inf")) == ARG
+    assert _fwd(lib, H=68) == SHAPE          # bf16 rows must be 16-byte multiples
+    assert _fwd(lib, H=4) == SHAPE
+    assert _fwd(lib, V=0) == SHAPE
+    assert _fwd(lib, N=-3) == SHAPE
+    assert _fwd(lib, hidden=None) == ARG
+    assert _fwd(lib, weight=FAKE + 8) == ARG  # misaligned for TMA
+    assert _fwd(lib, labels=FAKE + 4) == ARG
+    assert _fwd(lib, ws_size=1024) == WS
+    assert _fwd(lib, loss=None) == ARG
+    bad_bwd = lib.flce_backward(FAKE, FAKE, FAKE, FAKE, 64, 64, 512, -100, 0.0, 0, 0, None,
+                                float("nan"), None, FAKE, FAKE, FAKE,
+                                lib.flce_workspace_bytes(64, 64, 512, 0), None)
+    assert bad_bwd == ARG
+    assert lib.flce_get_status(None, None) == ARG
+
+
+def test_profile_api_host_side(lib):
+    ms = ctypes.c_double()
+    n = ctypes.c_int64()
+    assert lib.flce_profile_read(0, ctypes.byref(ms), ctypes.byref(n)) == 0
+    assert n.value == 0
+    assert lib.flce_profile_read(99, ctypes.byref(ms), ctypes.byref(n)) == 1
+    assert lib.flce_profile_enable(0) == 0

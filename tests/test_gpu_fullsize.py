@@ -1,0 +1,151 @@
+"""GPU parity at the full workload sizes, in the launch configuration the
+benchmark times.
+
+The V=32000 problem is compared in full against the float64 oracle.  For the
+larger ones the oracle's full-size values (every row's logsumexp and label
+logit, the loss, the counts) were written by tests/golden/make_oracle_fullsize.py,
+which calls only the oracle; dHidden and dWeight are compared on seeded
+samples of rows that the oracle computes one by one.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import flce_inputs as fi
+import lm_head_linear_tmem_b200 as flce
+import oracle
+from tests import _gpu as G
+
+pytestmark = pytest.mark.gpu
+IGN = fi.IGNORE_INDEX
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def golden(name):
+    path = os.path.join(GOLDEN, f"oracle_{name}.npz")
+    if not os.path.exists(path):
+        pytest.fail(f"missing {path}: run tests/golden/make_oracle_fullsize.py")
+    return np.load(path)
+
+
+def device_inputs(inp):
+    return (G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
+            G.labels_tensor(inp.labels))
+
+
+def sample_rows(labels, k, seed):
+    g = np.random.default_rng(seed)
+    N = len(labels)
+    rows = set(g.choice(N, size=k, replace=False).tolist())
+    rows |= {0, N - 1}
+    ign = np.nonzero(labels == IGN)[0]
+    if len(ign):
+        rows |= set(g.choice(ign, size=min(4, len(ign)), replace=False).tolist())
+    return np.array(sorted(rows))
+
+
+def sample_vocab(labels, V, k, seed):
+    g = np.random.default_rng(seed + 1)
+    rows = set(g.choice(V, size=k, replace=False).tolist())
+    valid = labels[labels != IGN]
+    counts = np.bincount(valid, minlength=V)
+    rows |= set(np.argsort(counts)[-6:].tolist())  # the most frequent labels
+    rows |= {0, V - 1}
+    return np.array(sorted(rows))
+
+
+def test_v32k_mean_full_compare():
+    inp = fi.make_inputs("v32k_mean")
+    w = inp.workload
+    h, W, y = device_inputs(inp)
+    f = flce.forward(h, W, y, IGN, w.softcap, w.reduction, check_status=True)
+    dh, dw = flce.backward(h, W, y, f.lse, softcap=w.softcap, reduction=w.reduction,
+                           check_status=True)
+    assert int(f.num_tokens.item()) == 0  # 'mean' returns num_tokens = 0
+    H64, W64 = inp.hidden.astype(np.float64), inp.weight.astype(np.float64)
+    rf = oracle.forward(H64, W64, inp.labels, IGN, w.softcap, w.reduction)
+    G.check_loss(f.loss.item(), rf["loss"])
+    assert np.max(np.abs(f.lse.cpu().numpy() - rf["lse"])) <= G.LSE_ATOL
+    rb = oracle.backward(H64, W64, inp.labels, IGN, w.softcap, w.reduction)
+    dh_np, dw_np = dh.cpu().numpy(), dw.cpu().numpy()
+    assert np.all(dh_np[inp.labels == IGN] == 0.0)
+    assert G.rel_l2(dh_np, rb["d_hidden"]) <= G.GRAD_RL2
+    assert G.rel_l2(dw_np, rb["d_weight"]) <= G.GRAD_RL2
+
+
+def _check_sampled(inp, gold, lse_gpu, dh, dw, g, seed):
+    w = inp.workload
+    H64, W64 = inp.hidden.astype(np.float64), inp.weight.astype(np.float64)
+    assert np.max(np.abs(lse_gpu - gold["lse"])) <= G.LSE_ATOL
+    ign = inp.labels == IGN
+    assert np.all(dh[ign] == 0.0)
+    assert np.all(np.isfinite(dh))
+    rows = sample_rows(inp.labels, 40, seed)
+    ref_dh = oracle.d_hidden_rows(H64, W64, inp.labels, rows, g, IGN, w.softcap)
+    assert G.rel_l2(dh[rows], ref_dh) <= G.GRAD_RL2
+    vrows = sample_vocab(inp.labels, w.V, 40, seed)
+    ref_dw = oracle.d_weight_rows(H64, W64, inp.labels, vrows, gold["lse"], g, IGN, w.softcap)
+    got_dw = dw[vrows]
+    assert np.all(np.isfinite(got_dw))
+    assert G.rel_l2(got_dw, ref_dw) <= G.GRAD_RL2
+
+
+@pytest.mark.parametrize("name", ["v131k_zipf", "v256k_softcap"])
+def test_fullsize_sampled(name):
+    gold = golden(name)
+    inp = fi.make_inputs(name)
+    w = inp.workload
+    h, W, y = device_inputs(inp)
+    f = flce.forward(h, W, y, IGN, w.softcap, w.reduction, check_status=True)
+    dh, dw = flce.backward(h, W, y, f.lse, softcap=w.softcap, reduction=w.reduction,
+                           check_status=True)
+    torch.cuda.synchronize()
+    assert int(f.num_tokens.item()) == int(gold["num_tokens"])
+    G.check_loss(f.loss.item(), float(gold["loss"]))
+    dh_np = dh.cpu().numpy()
+    del dh
+    dw_np = dw.cpu().numpy()
+    del dw
+    _check_sampled(inp, gold, f.lse.cpu().numpy(), dh_np, dw_np, 1.0, seed=sum(map(ord, name)))
+
+
+def test_microbatch_token_weighted_scale():
+    """4 micro-batches of 4096 tokens, micro-batch 1 all ignored; 'sum' with
+    grad_scale = 1 / sum_k n_k; dWeight accumulated over the micro-batches."""
+    gold = golden("microbatch")
+    inp = fi.make_inputs("microbatch")
+    w = inp.workload
+    h, W, y = device_inputs(inp)
+    n_tot = int(gold["num_valid"])
+    gs = 1.0 / n_tot
+    dw_acc = torch.zeros(w.V, w.H, dtype=torch.float32, device="cuda")
+    dh_all = torch.empty(w.N, w.H, dtype=torch.float32, device="cuda")
+    lse_all = torch.empty(w.N, dtype=torch.float32, device="cuda")
+    total = 0.0
+    ntok = 0
+    ws = flce.alloc_workspace(w.N // w.microbatches, w.H, w.V, torch.bfloat16, "cuda")
+    for k, sl in enumerate(inp.microbatch_slices()):
+        f = flce.forward(h[sl], W, y[sl], IGN, 0.0, "sum", workspace=ws, check_status=True)
+        dh, dw = flce.backward(h[sl], W, y[sl], f.lse, grad_scale=gs, workspace=ws,
+                               check_status=True)
+        lk = f.loss.item()
+        nk = int(f.num_tokens.item())
+        assert nk == int(gold["mb_count"][k])
+        G.check_loss(lk, float(gold["mb_loss"][k]))
+        if k == w.empty_microbatch:
+            assert lk == 0.0 and nk == 0
+            assert bool(torch.all(dh == 0)) and bool(torch.all(dw == 0))
+        assert bool(torch.isfinite(dw).all())
+        total += lk
+        ntok += nk
+        dw_acc += dw
+        dh_all[sl] = dh
+        lse_all[sl] = f.lse
+        del dw
+    assert ntok == n_tot
+    G.check_loss(total, float(gold["loss"]))
+    torch.cuda.synchronize()
+    _check_sampled(inp, gold, lse_all.cpu().numpy(), dh_all.cpu().numpy(),
+                   dw_acc.cpu().numpy(), gs, seed=5)

@@ -1,0 +1,159 @@
+"""GPU parity of the CUDA path (through the C ABI) against the float64 oracle
+on small problems that span several tiles, ragged tails and several backward
+chunks, plus the edge cases of the method."""
+import numpy as np
+import pytest
+import torch
+
+import flce_inputs as fi
+import lm_head_linear_tmem_b200 as flce
+import oracle
+from tests import _gpu as G
+
+pytestmark = pytest.mark.gpu
+IGN = fi.IGNORE_INDEX
+
+
+def run(h, w, y, softcap, reduction, grad_scale=1.0, grad_output=None, ignore_index=IGN):
+    f = flce.forward(h, w, y, ignore_index, softcap, reduction, check_status=True)
+    dh, dw = flce.backward(h, w, y, f.lse, grad_output=grad_output, grad_scale=grad_scale,
+                           ignore_index=ignore_index, softcap=softcap, reduction=reduction,
+                           check_status=True)
+    torch.cuda.synchronize()
+    return dict(loss=f.loss.item(), ntok=int(f.num_tokens.item()), lse=f.lse.cpu().numpy(),
+                dh=dh.cpu().numpy(), dw=dw.cpu().numpy(), loss_dtype=f.loss.dtype)
+
+
+def compare(got, hidden, weight, labels, softcap, reduction, grad_scale=1.0, grad_output=1.0,
+            ignore_index=IGN):
+    rf = oracle.forward(hidden, weight, labels, ignore_index, softcap, reduction)
+    rb = oracle.backward(hidden, weight, labels, ignore_index, softcap, reduction,
+                         grad_output=grad_output, grad_scale=grad_scale)
+    assert got["loss_dtype"] == torch.float32
+    assert got["ntok"] == rf["num_tokens"]
+    G.check_loss(got["loss"], rf["loss"])
+    assert np.max(np.abs(got["lse"] - rf["lse"])) <= G.LSE_ATOL
+    ign = labels == ignore_index
+    assert np.all(got["dh"][ign] == 0.0), "ignored rows must get exact zero gradient"
+    assert np.all(np.isfinite(got["dh"])) and np.all(np.isfinite(got["dw"]))
+    assert G.rel_l2(got["dh"], rb["d_hidden"]) <= G.GRAD_RL2
+    assert G.rel_l2(got["dw"], rb["d_weight"]) <= G.GRAD_RL2
+    return rf, rb
+
+
+def test_tiny_bf16_tensor_core_path():
+    inp = fi.make_inputs("tiny")
+    w = inp.workload
+    got = run(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
+              G.labels_tensor(inp.labels), w.softcap, w.reduction)
+    compare(got, inp.hidden, inp.weight, inp.labels, w.softcap, w.reduction)
+
+
+def test_tiny_fp32_cuda_core_path():
+    inp = fi.make_inputs("tiny", keep_raw=True)
+    w = inp.workload
+    got = run(G.f32_tensor(inp.hidden_raw), G.f32_tensor(inp.weight_raw),
+              G.labels_tensor(inp.labels), w.softcap, w.reduction)
+    rf, rb = compare(got, inp.hidden_raw, inp.weight_raw, inp.labels, w.softcap, w.reduction)
+    # fp32 end to end: much tighter than the bf16-operand bar
+    assert G.rel_l2(got["dh"], rb["d_hidden"]) <= 1e-5
+    assert G.rel_l2(got["dw"], rb["d_weight"]) <= 1e-5
+
+
+@pytest.mark.parametrize("softcap", [0.0, 5.0])
+@pytest.mark.parametrize("reduction", ["sum", "mean"])
+def test_ragged_multi_tile(softcap, reduction):
+    # N, V not multiples of the 128 x 256 tile; H not a multiple of the 64 K-block
+    inp = G.small_inputs(N=300, H=200, V=1000, seed=7, n_ign=60, w_std=0.2)
+    go = torch.tensor(0.75, device="cuda")
+    got = run(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
+              G.labels_tensor(inp.labels), softcap, reduction, grad_scale=1.3, grad_output=go)
+    compare(got, inp.hidden, inp.weight, inp.labels, softcap, reduction, grad_scale=1.3,
+            grad_output=0.75)
+
+
+@pytest.mark.parametrize("softcap", [0.0, 3.0])
+def test_several_backward_chunks(softcap):
+    # 2 token chunks x 2 vocab chunks: exercises the TMA reduce-add accumulation
+    inp = G.small_inputs(N=4500, H=136, V=9000, seed=8, n_ign=450, w_std=0.1)
+    got = run(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
+              G.labels_tensor(inp.labels), softcap, "sum", grad_scale=1.0 / 4050)
+    compare(got, inp.hidden, inp.weight, inp.labels, softcap, "sum", grad_scale=1.0 / 4050)
+
+
+def test_all_ignored_gives_zero_not_nan():
+    inp = G.small_inputs(N=200, H=64, V=700, seed=9, n_ign=0)
+    y = np.full(200, IGN, dtype=np.int64)
+    for red in ("sum", "mean"):
+        got = run(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
+                  G.labels_tensor(y), 0.0, red)
+        assert got["loss"] == 0.0 and got["ntok"] == 0
+        assert np.all(got["dh"] == 0.0) and np.all(got["dw"] == 0.0)
+        assert np.all(np.isfinite(got["lse"]))
+
+
+def test_empty_batch():
+    w = torch.zeros(512, 64, dtype=torch.bfloat16, device="cuda")
+    h = torch.zeros(0, 64, dtype=torch.bfloat16, device="cuda")
+    y = torch.zeros(0, dtype=torch.int64, device="cuda")
+    f = flce.forward(h, w, y, check_status=True)
+    assert f.loss.item() == 0.0 and f.num_tokens.item() == 0
+    dh, dw = flce.backward(h, w, y, f.lse, check_status=True)
+    assert dh.shape == (0, 64) and torch.all(dw == 0)
+
+
+def test_single_token_and_ignore_index_inside_vocab():
+    inp = G.small_inputs(N=1, H=64, V=300, seed=10, n_ign=0)
+    got = run(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
+              G.labels_tensor(inp.labels), 0.0, "sum")
+    compare(got, inp.hidden, inp.weight, inp.labels, 0.0, "sum")
+    # an ignore_index that is a real vocab id: rows with that label are ignored
+    inp = G.small_inputs(N=257, H=64, V=300, seed=11, n_ign=0)
+    y = inp.labels.copy()
+    y[::3] = 7
+    got = run(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
+              G.labels_tensor(y), 0.0, "mean", ignore_index=7)
+    compare(got, inp.hidden, inp.weight, y, 0.0, "mean", ignore_index=7)
+
+
+def test_label_out_of_range_is_reported():
+    inp = G.small_inputs(N=130, H=64, V=300, seed=12, n_ign=0)
+    y = inp.labels.copy()
+    y[5] = 300  # == V
+    with pytest.raises(flce.FlceError) as e:
+        flce.forward(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
+                     G.labels_tensor(y), check_status=True)
+    assert e.value.status == 3
+    # the status is cleared by the next forward
+    flce.forward(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
+                 G.labels_tensor(inp.labels), check_status=True)
+
+
+def test_module_autograd_and_num_tokens_contract():
+    inp = G.small_inputs(N=256, H=128, V=640, seed=13, n_ign=40, w_std=0.1)
+    h = G.bf16_tensor(inp.hidden_bits).requires_grad_(True)
+    w = G.bf16_tensor(inp.weight_bits).requires_grad_(True)
+    y = G.labels_tensor(inp.labels)
+    n = int((inp.labels != IGN).sum())
+    for red in ("sum", "mean"):
+        mod = flce.FusedLinearCrossEntropy(ignore_index=IGN, logit_softcapping=2.0, reduction=red)
+        loss = mod(h.view(2, 128, 128), y.view(2, 128), w)
+        assert loss.dtype == torch.float32
+        assert int(mod.num_tokens) == (n if red == "sum" else 0)
+        h.grad = None
+        w.grad = None
+        loss.backward()
+        rb = oracle.backward(inp.hidden, inp.weight, inp.labels, IGN, 2.0, red)
+        assert G.rel_l2(h.grad.float().cpu().numpy().reshape(256, 128), rb["d_hidden"]) < 5e-3
+        assert G.rel_l2(w.grad.float().cpu().numpy(), rb["d_weight"]) < 5e-3
+
+
+def test_repeated_calls_are_deterministic():
+    inp = G.small_inputs(N=4200, H=128, V=8500, seed=14, n_ign=100)
+    args = (G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
+            G.labels_tensor(inp.labels), 0.0, "sum")
+    a = run(*args)
+    b = run(*args)
+    assert a["loss"] == b["loss"]
+    assert np.array_equal(a["lse"], b["lse"])
+    assert np.array_equal(a["dh"], b["dh"]) and np.array_equal(a["dw"], b["dw"])
