@@ -117,6 +117,39 @@ flce_status flce_backward(const void* hidden, const void* weight, const int64_t*
                           float* d_hidden, float* d_weight, void* workspace,
                           size_t workspace_bytes, void* stream);
 
+/* Size of the library-owned device buffer behind flce_forward_noalloc. */
+#define FLCE_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/* Forward that allocates nothing and takes no workspace.  The pages have no
+ * counterpart to this entry point; it exists for callers that cannot allocate
+ * device memory at all: op/plugin interfaces that hand a kernel only its input
+ * and output buffers with no allocator, and programs that reserve the whole
+ * device memory in their own pool at start-up, where an extra cudaMalloc
+ * either fails or synchronises the device.
+ *
+ * Same arguments and results as flce_forward, minus the workspace.  Its
+ * scratch (per-vocab-tile softmax partials, label logits, loss partials) lives
+ * in one static __device__ buffer of FLCE_NOALLOC_SCRATCH_BYTES that every
+ * device which loads this library keeps until the process exits.
+ *  - Sizes whose forward scratch exceeds that buffer (about
+ *    8 * N * ceil(V / 256) bytes for bf16) return FLCE_ERR_SHAPE and launch
+ *    nothing; flce_forward with a caller workspace has no such limit.
+ *  - The first call on each device looks the buffer's device address up
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Every call on a device shares the one buffer, and the buffer keeps the
+ *    last call's contents (the call clears the part that must start at zero).
+ *    Calls whose kernels overlap on the GPU (different streams, or several
+ *    host threads) race on it: order them on one stream.
+ *  - status: optional device uint32[1]; receives the asynchronous error bits of
+ *    this call (1 = label outside [0, V) and not ignore_index, 2 = a bounded
+ *    pipeline wait ran out), 0 if none.  NULL skips it.
+ * It never calls cudaMalloc, cudaFree or any allocating library routine. */
+flce_status flce_forward_noalloc(const void* hidden, const void* weight, const int64_t* labels,
+                                 int64_t N, int64_t H, int64_t V, int64_t ignore_index,
+                                 float softcap, int32_t reduction, int32_t dtype, float* loss,
+                                 int64_t* num_tokens, float* lse, uint32_t* status, void* stream);
+
 /* Synchronise `stream`, then return the first asynchronous error recorded in
  * the workspace since the last flce_forward (FLCE_OK if none). */
 flce_status flce_get_status(const void* workspace, void* stream);

@@ -34,6 +34,8 @@ SIGNATURES = {
     "flce_backward": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32,
                               c_i32, c_i32, c_vp, c_f32, c_vp, c_vp, c_vp, c_vp, c_size,
                               c_vp]),
+    "flce_forward_noalloc": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32,
+                                     c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "flce_get_status": (c_i32, [c_vp, c_vp]),
     "flce_status_string": (ctypes.c_char_p, [c_i32]),
     "flce_version": (c_i32, []),

@@ -634,3 +634,84 @@ flce_status flce_profile_read(int32_t kind, double* total_ms, int64_t* launches)
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- no-alloc forward
+// flce_forward_noalloc: the bf16 / fp32 forward of flce_forward with its
+// scratch in a static device buffer instead of a caller workspace, for callers
+// that cannot allocate device memory (see include/flce.h).
+namespace flce {
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FLCE_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[64] = {};
+
+// Device address of g_noalloc_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device with that device current.
+flce_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= 64) return FLCE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return FLCE_OK;
+}
+
+}  // namespace
+}  // namespace flce
+
+extern "C" flce_status flce_forward_noalloc(const void* hidden, const void* weight,
+                                            const int64_t* labels, int64_t N, int64_t H,
+                                            int64_t V, int64_t ignore_index, float softcap,
+                                            int32_t reduction, int32_t dtype, float* loss,
+                                            int64_t* num_tokens, float* lse, uint32_t* status,
+                                            void* stream) {
+  if (reduction != FLCE_SUM && reduction != FLCE_MEAN) return FLCE_ERR_ARG;
+  if (dtype != FLCE_BF16 && dtype != FLCE_FP32) return FLCE_ERR_ARG;
+  if (!(softcap >= 0.f) || !(softcap < INFINITY)) return FLCE_ERR_ARG;
+  if (N < 0 || V < 1 || H < 8 || N > kMaxDim || V > kMaxDim || H > kMaxDim) return FLCE_ERR_SHAPE;
+  if (dtype == FLCE_BF16 && (H % 8) != 0) return FLCE_ERR_SHAPE;
+  if (dtype == FLCE_FP32 && H > kSimtMaxH) return FLCE_ERR_SHAPE;
+  if (N > 0 && (hidden == nullptr || labels == nullptr || lse == nullptr)) return FLCE_ERR_ARG;
+  if (weight == nullptr || loss == nullptr || num_tokens == nullptr) return FLCE_ERR_ARG;
+  if (!aligned16(hidden) || !aligned16(weight)) return FLCE_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(labels) & 7u) != 0) return FLCE_ERR_ARG;
+  // the forward's scratch must fit the static buffer
+  if (fwd_layout(N, V, dtype == FLCE_BF16).end > FLCE_NOALLOC_SCRATCH_BYTES) return FLCE_ERR_SHAPE;
+  DevInfo* d = nullptr;
+  flce_status s = device_info(&d);
+  if (s != FLCE_OK) return s;
+  void* ws = nullptr;
+  s = noalloc_scratch(&ws);
+  if (s != FLCE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // status word and n_valid start at zero
+  cudaError_t e = cudaMemsetAsync(ws, 0, 16, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (N == 0) {
+    if ((e = cudaMemsetAsync(loss, 0, sizeof(float), st)) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaMemsetAsync(num_tokens, 0, sizeof(int64_t), st)) != cudaSuccess)
+      return cuda_fail(e);
+  } else {
+    s = (dtype == FLCE_BF16)
+            ? forward_bf16(d, hidden, weight, labels, N, H, V, ignore_index, softcap, reduction,
+                           loss, num_tokens, lse, ws, st)
+            : forward_fp32(d, hidden, weight, labels, N, H, V, ignore_index, softcap, reduction,
+                           loss, num_tokens, lse, ws, st);
+    if (s != FLCE_OK) return s;
+  }
+  if (status != nullptr) {
+    e = cudaMemcpyAsync(status, ws, sizeof(uint32_t), cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return FLCE_OK;
+}
