@@ -17,7 +17,7 @@ def test_tiny_is_deterministic_and_quantised():
 
 
 def test_label_recipes():
-    for name, w in fi.WORKLOADS.items():
+    for name, w in fi.WORKLOADS.items():  # includes the profiling-size problem
         y = fi._draw_labels(w)
         assert y.shape == (w.N,) and y.dtype == np.int64
         valid = y != fi.IGNORE_INDEX
