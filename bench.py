@@ -40,15 +40,15 @@ import flce_inputs as fi  # noqa: E402
 METRIC = "FLCE fwd+bwd tokens/s at V=131072; % of B200 dense bf16 tensor peak"
 UNIT = "tokens/s"
 WORKLOAD = "v131k_zipf"
-KIND_NAMES = ["fwd_gemm_softmax_stats", "fwd_merge_loss", "bwd_dz_gemm", "bwd_dhidden_gemm",
-              "bwd_dweight_gemm", "helper", "fp32_simt"]
+KIND_NAMES = ["fwd_gemm_softmax_stats", "fwd_merge_loss", "bwd_dz_gemm", "bwd_dhidden_dweight_gemm",
+              "unused", "helper", "fp32_simt"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
 def parse_args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["own", "reference"], default="own")
     p.add_argument("--workload", default=WORKLOAD)
@@ -82,7 +82,7 @@ class ClockSampler:
         try:
             self.tmp = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
             cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                   "-lms", "200"]
+                   "-lms", "100"]
             if self.uuid:
                 cmd += ["-i", self.uuid]
             self.proc = subprocess.Popen(cmd, stdout=self.tmp, stderr=subprocess.DEVNULL)
@@ -256,34 +256,23 @@ def run_own(args, rank, world, local_rank):
     except Exception:
         uuid = None
 
-    # ---- device-resident timing (the headline value)
+    # ---- device-resident timing (the headline value): K steps, no per-kernel events
     barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(uuid)
     sampler.start()
-    lib.flce_profile_enable(1)
-    for k in range(len(KIND_NAMES)):  # drop records of the warm-up
-        lib.flce_profile_read(k, ctypes.byref(ctypes.c_double()), ctypes.byref(ctypes.c_int64()))
-    launches0 = lib.flce_launch_count()
     st = torch.cuda.current_stream()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    launches0 = lib.flce_launch_count()
     e0.record(st)
     for _ in range(args.steps):
         step()
     e1.record(st)
     torch.cuda.synchronize()
     launches = lib.flce_launch_count() - launches0
-    lib.flce_profile_enable(0)
     clocks = sampler.stop()
     ms = e0.elapsed_time(e1)
-    kinds = {}
-    for k, name in enumerate(KIND_NAMES):
-        t = ctypes.c_double()
-        n = ctypes.c_int64()
-        lib.flce_profile_read(k, ctypes.byref(t), ctypes.byref(n))
-        if n.value:
-            kinds[name] = {"ms_total": t.value, "launches": n.value}
     barrier()
     if world > 1:
         tt = torch.tensor([ms], dtype=torch.float64, device=dev)
@@ -291,6 +280,28 @@ def run_own(args, rank, world, local_rank):
         ms = float(tt.item())
     ms_step = ms / args.steps
     value = world * N * args.steps / (ms / 1e3)
+
+    # ---- per-kernel accounting: the same K steps again, with a CUDA event pair
+    # recorded by the library around every kernel it launches (on this stream)
+    lib.flce_profile_enable(1)
+    for k in range(len(KIND_NAMES)):  # drop anything recorded before
+        lib.flce_profile_read(k, ctypes.byref(ctypes.c_double()), ctypes.byref(ctypes.c_int64()))
+    torch.cuda.synchronize()
+    e0.record(st)
+    for _ in range(args.steps):
+        step()
+    e1.record(st)
+    torch.cuda.synchronize()
+    lib.flce_profile_enable(0)
+    ms_prof = e0.elapsed_time(e1)
+    kinds = {}
+    for k, name in enumerate(KIND_NAMES):
+        t = ctypes.c_double()
+        n = ctypes.c_int64()
+        lib.flce_profile_read(k, ctypes.byref(t), ctypes.byref(n))
+        if n.value:
+            kinds[name] = {"ms_total": t.value, "launches": n.value,
+                           "share": t.value / ms_prof if ms_prof > 0 else None}
 
     # ---- end to end through the API with host buffers
     e2e_steps = args.e2e_steps or max(3, args.steps // 2)
@@ -323,8 +334,9 @@ def run_own(args, rank, world, local_rank):
     peaks, peak_src = load_peaks()
     flops_step = w.flops_per_step
     # the dominant kernel (largest device time) and its roofline
+    # FLOP per step of each kernel kind (summed over its launches)
     credited = {"fwd_gemm_softmax_stats": 2.0 * N * H * V, "bwd_dz_gemm": 2.0 * N * H * V,
-                "bwd_dhidden_gemm": 2.0 * N * H * V, "bwd_dweight_gemm": 2.0 * N * H * V}
+                "bwd_dhidden_dweight_gemm": 4.0 * N * H * V}
     dom = max(kinds, key=lambda k: kinds[k]["ms_total"]) if kinds else None
     roofline = None
     if dom in credited:
@@ -359,6 +371,7 @@ def run_own(args, rank, world, local_rank):
                             "peak_source": peak_src},
         "roofline": roofline,
         "kernels": kinds,
+        "kernels_region_ms_per_step": ms_prof / args.steps,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},

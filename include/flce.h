@@ -169,8 +169,8 @@ uint64_t flce_launch_count(void);
  * kind, the summed device time in milliseconds and the number of launches
  * since the last read of that kind, then forgets them.
  * Kinds: 0 forward GEMM+softmax stats, 1 forward merge/loss, 2 backward dZ
- * GEMM, 3 backward dHidden GEMM, 4 backward dWeight GEMM, 5 small helper
- * kernels, 6 fp32 CUDA-core path. */
+ * GEMM, 3 backward dHidden+dWeight GEMMs (one launch per chunk), 4 unused,
+ * 5 small helper kernels, 6 fp32 CUDA-core path. */
 flce_status flce_profile_enable(int32_t enable);
 flce_status flce_profile_read(int32_t kind, double* total_ms, int64_t* launches);
 

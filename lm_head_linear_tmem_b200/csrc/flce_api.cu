@@ -6,8 +6,9 @@
 // bf16 path, backward:  the [N, V] problem is cut into chunks of at most
 //                       kChunkTokens x kChunkVocab; per chunk
 //                         tc_gemm<DzEpi>    dZ block (bf16, in the workspace)
-//                         tc_gemm<StoreEpi> dHidden[chunk rows] (+)= dZ . W[chunk]
-//                         tc_gemm<StoreEpi> dWeight[chunk rows] (+)= dZ^T . hidden[chunk]
+//                         tc_gemm<StoreEpi> (one launch, two GEMMs)
+//                           dHidden[chunk rows] (+)= dZ . W[chunk]
+//                           dWeight[chunk rows] (+)= dZ^T . hidden[chunk]
 //                       The first chunk along the reduced dimension stores,
 //                       later ones TMA-reduce-add into the fp32 outputs.
 // fp32 path:            simt_fwd / simt_dh / simt_dw (CUDA cores).
@@ -20,6 +21,8 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <set>
+#include <utility>
 #include <vector>
 
 #include "../../include/flce.h"
@@ -45,7 +48,7 @@ flce_status cuda_fail(cudaError_t e) {
 
 // ---------------------------------------------------------------- profiling
 constexpr int kKinds = 7;
-enum Kind { kFwdGemm = 0, kFwdMerge = 1, kBwdDz = 2, kBwdDh = 3, kBwdDw = 4, kHelper = 5, kSimt = 6 };
+enum Kind { kFwdGemm = 0, kFwdMerge = 1, kBwdDz = 2, kBwdDhDw = 3, kHelper = 5, kSimt = 6 };
 
 struct ProfRec {
   int kind;
@@ -86,7 +89,6 @@ struct DevInfo {
   bool init = false;
   bool ok = false;
   int sms = 0;
-  bool attr_set[8] = {false, false, false, false, false, false, false, false};
 };
 std::mutex g_dev_mu;
 DevInfo g_dev[64];
@@ -183,10 +185,23 @@ Chunking chunking(int64_t N, int64_t V) {
   return c;
 }
 
+// Backward GEMM launches of one call (at most three per chunk), each with its
+// own dynamic tile counter in the workspace.
+int64_t bwd_launches(int64_t N, int64_t V) {
+  const Chunking c = chunking(N, V);
+  return 3 * ((N + c.tc - 1) / c.tc) * ((V + c.vc - 1) / c.vc);
+}
+
+// Backward workspace: header | tile counters | dZ block (1024-aligned).
+size_t bwd_counters_offset() { return kHeaderBytes; }
+size_t bwd_gblock_offset(int64_t N, int64_t V) {
+  return align_up(kHeaderBytes + 4 * static_cast<size_t>(bwd_launches(N, V)), 1024);
+}
+
 size_t bwd_bytes(int64_t N, int64_t V, bool bf16) {
   if (!bf16) return kHeaderBytes;
   const Chunking c = chunking(N, V);
-  return align_up(kHeaderBytes, 1024) + static_cast<size_t>(c.tc) * c.vc * 2 + 1024;
+  return bwd_gblock_offset(N, V) + static_cast<size_t>(c.tc) * c.vc * 2 + 1024;
 }
 
 size_t ws_bytes(int64_t N, int64_t V, bool bf16) {
@@ -196,6 +211,22 @@ size_t ws_bytes(int64_t N, int64_t V, bool bf16) {
 unsigned int* ws_status(void* ws) { return reinterpret_cast<unsigned int*>(ws); }
 long long* ws_nvalid(void* ws) {
   return reinterpret_cast<long long*>(reinterpret_cast<char*>(ws) + 8);
+}
+
+// Tile shape of the tensor-core GEMMs: 2 = CTA pairs with 256 x 256 tiles
+// (default), 1 = single CTAs with 128 x 256 tiles.  FLCE_CTA_GROUP=1 selects
+// the latter (read at every call).
+int cta_group() {
+  const char* s = std::getenv("FLCE_CTA_GROUP");
+  return (s != nullptr && std::atoi(s) == 1) ? 1 : 2;
+}
+
+// Backward chunk schedule: the dHidden and dWeight GEMMs of a chunk share one
+// launch (default; tiles handed out dynamically, the long dHidden tiles
+// first), or FLCE_BWD_FUSE=0 gives each its own launch (read at every call).
+bool bwd_fuse_dhdw() {
+  const char* s = std::getenv("FLCE_BWD_FUSE");
+  return !(s != nullptr && std::atoi(s) == 0);
 }
 
 unsigned long long timeout_ns() {
@@ -230,29 +261,102 @@ flce_status check_common(const void* hidden, const void* weight, const int64_t* 
   return FLCE_OK;
 }
 
+// Opt a kernel in to `bytes` of dynamic shared memory, once per (device, kernel).
+std::mutex g_attr_mu;
+std::set<std::pair<int, const void*>> g_attr_done;
+
 template <class Kern>
-cudaError_t set_smem_attr(DevInfo* d, int slot, Kern k, size_t bytes) {
-  if (d->attr_set[slot]) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(bytes));
-  if (e == cudaSuccess) d->attr_set[slot] = true;
+cudaError_t set_smem_attr(DevInfo*, int, Kern k, size_t bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const auto key = std::make_pair(dev, reinterpret_cast<const void*>(k));
+  {
+    std::lock_guard<std::mutex> lk(g_attr_mu);
+    if (g_attr_done.count(key)) return cudaSuccess;
+  }
+  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e == cudaSuccess) {
+    std::lock_guard<std::mutex> lk(g_attr_mu);
+    g_attr_done.insert(key);
+  }
   return e;
 }
 
-// Kernel instantiation slots for the shared-memory attribute cache.
+// Kernel instantiation slots for the shared-memory attribute cache (x2: CTA group).
 enum Slot { kSlotFwd = 0, kSlotFwdCap, kSlotDz, kSlotDzCap, kSlotDh, kSlotDw, kSlotSimtDh, kSlotSimtDw };
 
-template <class Epi, bool kAMn, bool kBMn>
-cudaError_t run_gemm(DevInfo* d, int slot, int kind, const CUtensorMap& a, const CUtensorMap& b,
-                     const CUtensorMap& out, const GemmArgs& g, const typename Epi::Params& ep,
-                     cudaStream_t st) {
-  auto k = tc_gemm_kernel<Epi, kAMn, kBMn>;
-  cudaError_t e = set_smem_attr(d, slot, k, kGemmSmemBytes);
+// One GEMM of a launch: operand / output tensor maps, output rows M (tiled by
+// 128 * kCG) and the rest of its GemmArgs.
+struct GemmProblem {
+  const CUtensorMap* a;
+  const CUtensorMap* b;
+  const CUtensorMap* out;
+  int64_t M;
+  GemmArgs g;
+};
+
+// One tensor-core launch over one GEMM (p1 == nullptr) or two independent
+// GEMMs with the same epilogue.  kCG = 2 launches clusters of two CTAs.
+template <class Epi, int kCG, bool kAMn0, bool kBMn0, bool kAMn1, bool kBMn1>
+cudaError_t run_gemm_cg(DevInfo* d, int slot, int kind, const GemmProblem& p0,
+                        const typename Epi::Params& ep0, const GemmProblem* p1,
+                        const typename Epi::Params& ep1, cudaStream_t st) {
+  using Cfg = TileCfg<kCG>;
+  auto k = tc_gemm_kernel<Epi, kCG, kAMn0, kBMn0, kAMn1, kBMn1>;
+  cudaError_t e = set_smem_attr(d, 2 * slot + (kCG - 1), k, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int tiles = g.m_tiles * g.n_tiles;
-  const int grid = std::max(1, std::min(tiles, d->sms));
-  return launch(kind, st, [&] { k<<<grid, kThreads, kGemmSmemBytes, st>>>(a, b, out, g, ep); });
+  GemmArgs g0 = p0.g;
+  g0.m_tiles = static_cast<int>((p0.M + Cfg::kUnitRows - 1) / Cfg::kUnitRows);
+  GemmArgs g1 = p1 ? p1->g : p0.g;
+  if (p1)
+    g1.m_tiles = static_cast<int>((p1->M + Cfg::kUnitRows - 1) / Cfg::kUnitRows);
+  else
+    g1.m_tiles = g1.n_tiles = 0;
+  const GemmProblem& q1 = p1 ? *p1 : p0;
+  const int tiles = g0.m_tiles * g0.n_tiles + g1.m_tiles * g1.n_tiles;
+  const int units = std::max(1, std::min(tiles, d->sms / kCG));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(units * kCG, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int nattr = 0;
+  if (kCG > 1) {
+    attr[nattr].id = cudaLaunchAttributeClusterDimension;
+    attr[nattr].val.clusterDim.x = kCG;
+    attr[nattr].val.clusterDim.y = 1;
+    attr[nattr].val.clusterDim.z = 1;
+    ++nattr;
+  }
+  if (g0.dep_wait != kDepNone) {
+    // may start while the previous kernel drains; it waits where it depends on it
+    attr[nattr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[nattr].val.programmaticStreamSerializationAllowed = 1;
+    ++nattr;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = nattr;
+  cudaError_t le = cudaSuccess;
+  cudaError_t e2 = launch(kind, st, [&] {
+    le = cudaLaunchKernelEx(&cfg, k, *p0.a, *p0.b, *p0.out, *q1.a, *q1.b, *q1.out, g0, g1, ep0,
+                            ep1);
+  });
+  return le != cudaSuccess ? le : e2;
 }
+
+template <class Epi, bool kAMn0, bool kBMn0, bool kAMn1 = false, bool kBMn1 = false>
+cudaError_t run_gemm(DevInfo* d, int slot, int kind, const GemmProblem& p0,
+                     const typename Epi::Params& ep0, const GemmProblem* p1,
+                     const typename Epi::Params& ep1, cudaStream_t st) {
+  if (cta_group() == 2)
+    return run_gemm_cg<Epi, 2, kAMn0, kBMn0, kAMn1, kBMn1>(d, slot, kind, p0, ep0, p1, ep1, st);
+  return run_gemm_cg<Epi, 1, kAMn0, kBMn0, kAMn1, kBMn1>(d, slot, kind, p0, ep0, p1, ep1, st);
+}
+
+// Rows of B (K-major) one CTA stages per K-block.
+uint32_t b_box_rows() { return static_cast<uint32_t>(BN / cta_group()); }
 
 // ---------------------------------------------------------------- forward
 flce_status forward_bf16(DevInfo* d, const void* hidden, const void* weight,
@@ -269,11 +373,10 @@ flce_status forward_bf16(DevInfo* d, const void* hidden, const void* weight,
 
   CUtensorMap ta, tb;
   if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hidden, H, N, H * 2, BK, BM) ||
-      !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, weight, H, V, H * 2, BK, BN))
+      !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, weight, H, V, H * 2, BK, b_box_rows()))
     return FLCE_ERR_CUDA;
 
   GemmArgs g{};
-  g.m_tiles = static_cast<int>((N + BM - 1) / BM);
   g.n_tiles = static_cast<int>((V + BN - 1) / BN);
   g.k_blocks = static_cast<int>((H + BK - 1) / BK);
   g.group_m = kGroupM;
@@ -283,14 +386,17 @@ flce_status forward_bf16(DevInfo* d, const void* hidden, const void* weight,
   g.timeout_ns = timeout_ns();
 
   cudaError_t e;
+  const GemmProblem prob{&ta, &tb, &ta, N, g};
   if (softcap > 0.f) {
     FwdStatsEpi<true>::Params ep{labels, static_cast<int>(N), static_cast<int>(V), softcap,
                                  1.0f / softcap, part_m, part_s, label_logit};
-    e = run_gemm<FwdStatsEpi<true>, false, false>(d, kSlotFwdCap, kFwdGemm, ta, tb, ta, g, ep, st);
+    e = run_gemm<FwdStatsEpi<true>, false, false>(d, kSlotFwdCap, kFwdGemm, prob, ep, nullptr,
+                                                  ep, st);
   } else {
     FwdStatsEpi<false>::Params ep{labels, static_cast<int>(N), static_cast<int>(V), 0.f, 0.f,
                                   part_m, part_s, label_logit};
-    e = run_gemm<FwdStatsEpi<false>, false, false>(d, kSlotFwd, kFwdGemm, ta, tb, ta, g, ep, st);
+    e = run_gemm<FwdStatsEpi<false>, false, false>(d, kSlotFwd, kFwdGemm, prob, ep, nullptr, ep,
+                                                   st);
   }
   if (e != cudaSuccess) return cuda_fail(e);
 
@@ -362,12 +468,18 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
                           float* d_hidden, float* d_weight, void* ws, cudaStream_t st) {
   const Chunking ck = chunking(N, V);
   char* w = static_cast<char*>(ws);
-  void* gbuf = w + align_up(kHeaderBytes, 1024);
+  void* gbuf = w + bwd_gblock_offset(N, V);
+  int* counters = reinterpret_cast<int*>(w + bwd_counters_offset());
+  int next_counter = 0;
+  {
+    const cudaError_t e = cudaMemsetAsync(counters, 0, 4 * bwd_launches(N, V), st);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
 
   CUtensorMap t_hid_k, t_hid_mn, t_w_k, t_w_mn, t_dh, t_dw;
   if (!make_map(&t_hid_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hidden, H, N, H * 2, BK, BM) ||
       !make_map(&t_hid_mn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hidden, H, N, H * 2, 64, BK) ||
-      !make_map(&t_w_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, weight, H, V, H * 2, BK, BN) ||
+      !make_map(&t_w_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, weight, H, V, H * 2, BK, b_box_rows()) ||
       !make_map(&t_w_mn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, weight, H, V, H * 2, 64, BK) ||
       !make_map(&t_dh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d_hidden, H, N, H * 4, 32, 32) ||
       !make_map(&t_dw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d_weight, H, V, H * 4, 32, 32))
@@ -394,7 +506,6 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
 
       // 1) dZ = f(hidden[t0:] . W[v0:]^T) -> bf16 block
       GemmArgs gz{};
-      gz.m_tiles = (rows + BM - 1) / BM;
       gz.n_tiles = (cols + BN - 1) / BN;
       gz.k_blocks = k_blocks_h;
       gz.group_m = kGroupM;
@@ -402,52 +513,61 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
       gz.b_off = static_cast<int>(v0);
       gz.status = ws_status(ws);
       gz.timeout_ns = tmo;
+      gz.tile_counter = counters + next_counter++;
+      // dZ overwrites the block the previous chunk's dHidden/dWeight GEMMs read:
+      // its main loop may start early, its first store waits for them
+      gz.dep_wait = (t0 > 0 || v0 > 0) ? kDepBeforeStores : kDepNone;
       cudaError_t e;
+      const GemmProblem pz{&t_hid_k, &t_w_k, &t_g_store, rows, gz};
       if (softcap > 0.f) {
         DzEpi<true>::Params ep{labels, lse, ignore_index, static_cast<int>(t0), rows,
                                static_cast<int>(v0), cols, softcap, 1.0f / softcap};
-        e = run_gemm<DzEpi<true>, false, false>(d, kSlotDzCap, kBwdDz, t_hid_k, t_w_k, t_g_store,
-                                                gz, ep, st);
+        e = run_gemm<DzEpi<true>, false, false>(d, kSlotDzCap, kBwdDz, pz, ep, nullptr, ep, st);
       } else {
         DzEpi<false>::Params ep{labels, lse, ignore_index, static_cast<int>(t0), rows,
                                 static_cast<int>(v0), cols, 0.f, 0.f};
-        e = run_gemm<DzEpi<false>, false, false>(d, kSlotDz, kBwdDz, t_hid_k, t_w_k, t_g_store,
-                                                 gz, ep, st);
+        e = run_gemm<DzEpi<false>, false, false>(d, kSlotDz, kBwdDz, pz, ep, nullptr, ep, st);
       }
       if (e != cudaSuccess) return cuda_fail(e);
 
       // 2) dHidden[t0:t0+rows] (+)= dZ . W[v0:v0+cols]
       GemmArgs gh{};
-      gh.m_tiles = (rows + BM - 1) / BM;
       gh.n_tiles = n_tiles_h;
       gh.k_blocks = (cols + BK - 1) / BK;
       gh.group_m = kGroupM;
       gh.a_off = 0;
       gh.b_off = static_cast<int>(v0);
-      gh.a_mn_extent = 0;
-      gh.b_mn_extent = static_cast<int>(H);
       gh.status = ws_status(ws);
       gh.timeout_ns = tmo;
+      gh.tile_counter = counters + next_counter++;
+      gh.dep_wait = kDepBeforeLoads;  // reads the dZ block written just before
       StoreEpi::Params eh{static_cast<int>(t0), v0 > 0 ? 1 : 0, static_cast<int>(H),
                           static_cast<int>(N), grad_output, grad_scale, n_valid, mean};
-      e = run_gemm<StoreEpi, false, true>(d, kSlotDh, kBwdDh, t_g_k, t_w_mn, t_dh, gh, eh, st);
-      if (e != cudaSuccess) return cuda_fail(e);
 
       // 3) dWeight[v0:v0+cols] (+)= dZ^T . hidden[t0:t0+rows]
       GemmArgs gw{};
-      gw.m_tiles = (cols + BM - 1) / BM;
       gw.n_tiles = n_tiles_h;
       gw.k_blocks = (rows + BK - 1) / BK;
       gw.group_m = kGroupM;
       gw.a_off = 0;
       gw.b_off = static_cast<int>(t0);
-      gw.a_mn_extent = cols;
-      gw.b_mn_extent = static_cast<int>(H);
       gw.status = ws_status(ws);
       gw.timeout_ns = tmo;
+      gw.tile_counter = counters + next_counter++;
+      gw.dep_wait = kDepBeforeLoads;
       StoreEpi::Params ew{static_cast<int>(v0), t0 > 0 ? 1 : 0, static_cast<int>(H),
                           static_cast<int>(V), grad_output, grad_scale, n_valid, mean};
-      e = run_gemm<StoreEpi, true, true>(d, kSlotDw, kBwdDw, t_g_mn, t_hid_mn, t_dw, gw, ew, st);
+
+      const GemmProblem ph{&t_g_k, &t_w_mn, &t_dh, rows, gh};
+      const GemmProblem pw{&t_g_mn, &t_hid_mn, &t_dw, cols, gw};
+      if (bwd_fuse_dhdw()) {
+        // 2) + 3) in one launch: the dWeight tiles fill the dHidden grid's last wave
+        e = run_gemm<StoreEpi, false, true, true, true>(d, kSlotDh, kBwdDhDw, ph, eh, &pw, ew, st);
+      } else {
+        e = run_gemm<StoreEpi, false, true>(d, kSlotDh, kBwdDhDw, ph, eh, nullptr, eh, st);
+        if (e == cudaSuccess)
+          e = run_gemm<StoreEpi, true, true>(d, kSlotDw, kBwdDhDw, pw, ew, nullptr, ew, st);
+      }
       if (e != cudaSuccess) return cuda_fail(e);
     }
   }
@@ -463,9 +583,9 @@ flce_status backward_fp32(DevInfo* d, const void* hidden, const void* weight,
   const int mean = reduction == FLCE_MEAN;
   const size_t sh_dh = (2 * static_cast<size_t>(h) + kSimtChunk) * sizeof(float);
   const size_t sh_dw = (2 * static_cast<size_t>(h) + kSimtThreads) * sizeof(float);
-  cudaError_t e = set_smem_attr(d, kSlotSimtDh, simt_dh_kernel, 2 * kSimtMaxH * 4 + kSimtChunk * 4);
+  cudaError_t e = set_smem_attr(d, 2 * kSlotSimtDh, simt_dh_kernel, 2 * kSimtMaxH * 4 + kSimtChunk * 4);
   if (e != cudaSuccess) return cuda_fail(e);
-  e = set_smem_attr(d, kSlotSimtDw, simt_dw_kernel, 2 * kSimtMaxH * 4 + kSimtThreads * 4);
+  e = set_smem_attr(d, 2 * kSlotSimtDw, simt_dw_kernel, 2 * kSimtMaxH * 4 + kSimtThreads * 4);
   if (e != cudaSuccess) return cuda_fail(e);
   if (n > 0) {
     e = launch(kSimt, st, [&] {

@@ -2,13 +2,22 @@
 //
 // One CTA per SM (192 threads, ~225 KB shared memory, all 512 TMEM columns).
 // Warp roles:
-//   warp 0  TMA producer   (one thread): K-blocks of A and B into a 4-stage ring
-//   warp 1  MMA issuer     (one thread): tcgen05.mma M=128 N=256 K=16, fp32 in TMEM;
+//   warp 0  TMA producer   (one thread): K-blocks of A and B into a stage ring
+//   warp 1  MMA issuer     (one thread): tcgen05.mma K=16 steps, fp32 in TMEM;
 //                                        two 256-column accumulators so the
 //                                        epilogue of tile i overlaps the MMAs of i+1
 //   warps 2-5 epilogue     (128 threads, thread = accumulator row): tcgen05.ld
 //                                        then an operation-specific epilogue
-// Output tile 128 x 256, K-block 64 (one 128-byte swizzle row of bf16).
+// Two tile shapes (template parameter kCG, the CTA group):
+//   kCG = 1  one CTA computes a 128 x 256 tile (tcgen05.mma.cta_group::1,
+//            M=128 N=256), 4 stages of 48 KiB;
+//   kCG = 2  a cluster of two CTAs computes a 256 x 256 tile with one
+//            tcgen05.mma.cta_group::2 (M=256 N=256) issued by the pair's
+//            leader: each CTA stages its own 128 rows of A and 128 rows of B
+//            (32 KiB a stage, 6 stages) and holds its own 128 x 256
+//            accumulator rows in TMEM, so each SM moves half the operand bytes
+//            per FLOP of the 1-CTA shape.
+// K-block 64 (one 128-byte swizzle row of bf16).
 //
 // Operands may be K-major (row-major [rows, K], the usual "TN" GEMM) or
 // MN-major (row-major [K, rows]); both are staged with 128-byte swizzle and
@@ -17,9 +26,9 @@
 // The three epilogues implement the steps of the fused linear cross-entropy:
 //   FwdStatsEpi  softcap, per-row online max / sum of exp over the tile's 256
 //                vocab columns, label-logit capture (forward)
-//   DzEpi        softcap, dZ = g*(exp(L-lse) - onehot)*softcap' -> bf16 block
+//   DzEpi        softcap, dZ/g = (exp(L-lse) - onehot)*softcap' -> bf16 block
 //                of dZ in global memory via TMA store (backward)
-//   StoreEpi     fp32 tile -> TMA store or TMA reduce-add (dHidden, dWeight)
+//   StoreEpi     g * fp32 tile -> TMA store or TMA reduce-add (dHidden, dWeight)
 // The GEMM itself is the LM-head projection logits = hidden . weight^T
 // (NeMo AutoModel linear_ce API: lm_weight is [vocab, hidden]) and, in the
 // backward, dZ . weight and dZ^T . hidden.
@@ -32,20 +41,28 @@
 
 namespace flce {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BM = 128;  // accumulator rows held by one CTA
+constexpr int BN = 256;  // accumulator columns
 constexpr int BK = 64;
-constexpr int kStages = 4;
 constexpr int kABytes = BM * BK * 2;  // 16 KB
-constexpr int kBBytes = BN * BK * 2;  // 32 KB
-constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kEpiWarps = 4;
 constexpr int kStagingBuf = 4096;                 // 32 rows x 128 bytes
 constexpr int kStagingPerWarp = 2 * kStagingBuf;  // double buffered
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
-constexpr size_t kGemmSmemBytes =
-    1024 + static_cast<size_t>(kStages) * kStageBytes + kEpiWarps * kStagingPerWarp;
+
+template <int kCG>
+struct TileCfg {
+  static constexpr int kBRows = BN / kCG;  // B rows (N index) staged by one CTA
+  static constexpr int kBBytes = kBRows * BK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = kCG == 1 ? 4 : 6;
+  static constexpr int kUnitRows = BM * kCG;  // output rows of one tile
+  static constexpr size_t kSmemBytes =
+      1024 + static_cast<size_t>(kStages) * kStageBytes + kEpiWarps * kStagingPerWarp;
+};
+
+constexpr int kRing = 8;  // tile indices in flight between the fetcher and the other roles
 
 constexpr uint32_t kStatusLabelRange = 1u;
 constexpr uint32_t kStatusTimeout = 2u;
@@ -54,17 +71,24 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 struct GemmArgs {
-  int m_tiles;
-  int n_tiles;
+  int m_tiles;    // tiles of kUnitRows output rows
+  int n_tiles;    // tiles of BN output columns
   int k_blocks;
   int group_m;    // tiles are walked in groups of group_m row-tiles (L2 reuse)
   int a_off;      // added to A's outer (row) TMA coordinate
   int b_off;      // added to B's outer (row) TMA coordinate
-  int a_mn_extent;  // MN-major A: extent of its inner (M) dimension
-  int b_mn_extent;  // MN-major B: extent of its inner (N) dimension
   unsigned int* status;
   unsigned long long timeout_ns;
+  int* tile_counter;  // zeroed device counter: tiles are handed out dynamically;
+                      // nullptr: static round-robin over the CTAs (or CTA pairs)
+  int dep_wait;       // what waits for the previous kernel on the stream (launched
+                      // as a programmatic dependent): kDepNone, kDepBeforeLoads
+                      // (operands it produced), kDepBeforeStores (an output it reads)
 };
+
+constexpr int kDepNone = 0;
+constexpr int kDepBeforeLoads = 1;
+constexpr int kDepBeforeStores = 2;
 
 __device__ __forceinline__ void tile_coords(int tile, const GemmArgs& g, int& mb, int& nb) {
   const int per_group = g.group_m * g.n_tiles;
@@ -76,10 +100,12 @@ __device__ __forceinline__ void tile_coords(int tile, const GemmArgs& g, int& mb
   nb = r / gm;
 }
 
+// Hand the accumulator back to the MMA issuer: `tempty_bar` is the
+// shared::cluster address of the (leader CTA's) accumulator-empty barrier.
 __device__ __forceinline__ void release_tmem(uint32_t tempty_bar, int lane) {
   tc_fence_before();
   __syncwarp();
-  if (lane == 0) mbar_arrive(tempty_bar);
+  if (lane == 0) mbar_arrive_cluster(tempty_bar);
 }
 
 // Write 128 bytes (8 x 16 B) of row `lane` into a 32-row staging buffer laid
@@ -112,10 +138,10 @@ struct FwdStatsEpi {
     float* label_logit;  // [N]
   };
 
-  __device__ static void tile(const Params& p, const GemmArgs&, int mb, int nb, uint32_t taddr,
-                              int q, int lane, uint8_t*, const CUtensorMap*, uint32_t tempty,
-                              int&) {
-    const int row = mb * BM + q * 32 + lane;
+  __device__ static void tile(const Params& p, const GemmArgs&, int m_base, int nb,
+                              uint32_t taddr, int q, int lane, uint8_t*, const CUtensorMap*,
+                              uint32_t tempty, int&) {
+    const int row = m_base + q * 32 + lane;
     const bool row_ok = row < p.N;
     const int col0 = nb * BN;
     int y_local = -1;
@@ -183,11 +209,11 @@ struct DzEpi {
     float inv_softcap;
   };
 
-  __device__ static void tile(const Params& p, const GemmArgs&, int mb, int nb, uint32_t taddr,
-                              int q, int lane, uint8_t* stg, const CUtensorMap* out,
-                              uint32_t tempty, int& nstore) {
+  __device__ static void tile(const Params& p, const GemmArgs&, int m_base, int nb,
+                              uint32_t taddr, int q, int lane, uint8_t* stg,
+                              const CUtensorMap* out, uint32_t tempty, int& nstore) {
     // 64-column chunks whose store box starts inside the block (warp-uniform)
-    const int y0 = mb * BM + q * 32;
+    const int y0 = m_base + q * 32;
     const int rem = p.cols - nb * BN;
     const int nch = (y0 >= p.rows || rem <= 0) ? 0 : min(BN / 64, (rem + 63) / 64);
     if (nch == 0) {
@@ -277,11 +303,11 @@ struct StoreEpi {
     return g;
   }
 
-  __device__ static void tile(const Params& p, const GemmArgs&, int mb, int nb, uint32_t taddr,
-                              int q, int lane, uint8_t* stg, const CUtensorMap* out,
-                              uint32_t tempty, int& nstore) {
+  __device__ static void tile(const Params& p, const GemmArgs&, int m_base, int nb,
+                              uint32_t taddr, int q, int lane, uint8_t* stg,
+                              const CUtensorMap* out, uint32_t tempty, int& nstore) {
     // 32-column chunks whose store box starts inside the output (warp-uniform)
-    const int y = p.out_row0 + mb * BM + q * 32;
+    const int y = p.out_row0 + m_base + q * 32;
     const int rem = p.x_limit - nb * BN;
     const int nch = (y >= p.y_limit || rem <= 0) ? 0 : min(BN / 32, (rem + 31) / 32);
     if (nch == 0) {
@@ -323,17 +349,36 @@ __device__ __forceinline__ void record_timeout(const GemmArgs& g, volatile int* 
   if (g.status != nullptr) atomicOr(g.status, kStatusTimeout);
 }
 
-template <class Epi, bool kAMn, bool kBMn>
+template <int kCG>
+__device__ __forceinline__ void load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                        int32_t x, int32_t y) {
+  if constexpr (kCG == 1)
+    tma_load_2d(dst, map, bar, x, y);
+  else
+    tma_load_2d_pair(dst, map, bar, x, y);
+}
+
+// One launch runs the tiles of one GEMM, or of two independent GEMMs that
+// share the epilogue type (problem 0's tiles first, then problem 1's, so the
+// last wave of one is filled by the other).  Operand majors are per problem.
+template <class Epi, int kCG, bool kAMn0, bool kBMn0, bool kAMn1 = false, bool kBMn1 = false>
 __global__ void __launch_bounds__(kThreads, 1)
-    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmOut, const GemmArgs g,
-                   const typename Epi::Params ep) {
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+                   const __grid_constant__ CUtensorMap tmOut0, const __grid_constant__ CUtensorMap tmA1,
+                   const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmOut1,
+                   const GemmArgs g0, const GemmArgs g1, const typename Epi::Params ep0,
+                   const typename Epi::Params ep1) {
+  using Cfg = TileCfg<kCG>;
+  constexpr int kStages = Cfg::kStages;
   extern __shared__ uint8_t smem_dyn[];
   __shared__ __align__(8) uint64_t bar_full[kStages];
   __shared__ __align__(8) uint64_t bar_empty[kStages];
   __shared__ __align__(8) uint64_t bar_tfull[2];
   __shared__ __align__(8) uint64_t bar_tempty[2];
   __shared__ __align__(8) uint64_t bar_drain;
+  __shared__ __align__(8) uint64_t ring_full[kRing];
+  __shared__ __align__(8) uint64_t ring_empty[kRing];
+  __shared__ int tile_ring[kRing];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -342,6 +387,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_dyn + pad;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = (kCG == 1) ? 0u : cluster_ctarank();
+  const bool leader = (rank == 0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -350,74 +397,151 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&bar_tfull[a]), 1);
-      mbar_init(smem_u32(&bar_tempty[a]), kEpiWarps);
+      mbar_init(smem_u32(&bar_tempty[a]), kEpiWarps * kCG);
     }
     mbar_init(smem_u32(&bar_drain), 1);
+    // each tile index is read by: the MMA issuer and 4 epilogue warps of the
+    // leader, and the producer and 4 epilogue warps of the peer
+    for (int r = 0; r < kRing; ++r) {
+      mbar_init(smem_u32(&ring_full[r]), 1);
+      mbar_init(smem_u32(&ring_empty[r]), (1 + kEpiWarps) * kCG);
+    }
     abort_sh = 0;
     fence_mbar_init();
-    prefetch_tmap(&tmA);
-    prefetch_tmap(&tmB);
-    prefetch_tmap(&tmOut);
+    prefetch_tmap(&tmA0);
+    prefetch_tmap(&tmB0);
+    prefetch_tmap(&tmOut0);
+    if (g1.m_tiles > 0) {
+      prefetch_tmap(&tmA1);
+      prefetch_tmap(&tmB1);
+      prefetch_tmap(&tmOut1);
+    }
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(&tmem_base_sh), kTmemCols);
-    tmem_relinquish();
+    if constexpr (kCG == 1) {
+      tmem_alloc(smem_u32(&tmem_base_sh), kTmemCols);
+      tmem_relinquish();
+    } else {
+      tmem_alloc_pair(smem_u32(&tmem_base_sh), kTmemCols);
+      tmem_relinquish_pair();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (kCG == 1)
+    __syncthreads();
+  else
+    cluster_sync();  // the leader's barriers are initialised before the peer uses them
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_sh;
-  const int num_tiles = g.m_tiles * g.n_tiles;
+  // The next kernel on the stream may be scheduled as SMs free up; it waits
+  // for this one wherever it depends on it.
+  griddep_launch_dependents();
+  const int tiles0 = g0.m_tiles * g0.n_tiles;
+  const int num_tiles = tiles0 + g1.m_tiles * g1.n_tiles;
+  const int unit = blockIdx.x / kCG;  // CTA (kCG = 1) or CTA pair (kCG = 2)
+  const int n_units = gridDim.x / kCG;
   volatile int* abort_flag = &abort_sh;
+
+  // problem, its args and the tile's coordinates for global tile index t
+  auto locate = [&](int t, int& prob, int& mb, int& nb) {
+    prob = (t < tiles0) ? 0 : 1;
+    tile_coords(prob ? t - tiles0 : t, prob ? g1 : g0, mb, nb);
+  };
+
+  // ---- tile hand-out.  The leader's producer thread picks each next tile
+  // (an atomic on g0.tile_counter, or unit + k * n_units without one) and
+  // publishes it in a ring slot of both CTAs; every other role reads the
+  // same sequence from its own CTA's ring.  A value >= num_tiles ends it.
+  auto ring_publish = [&](int slot, uint32_t rph, int t) -> bool {
+    if (!mbar_wait(smem_u32(&ring_empty[slot]), rph ^ 1u, abort_flag, g0.timeout_ns)) return false;
+    tile_ring[slot] = t;
+    if constexpr (kCG == 2) {
+      const uint32_t peer_slot = mapa_shared(smem_u32(&tile_ring[slot]), 1);
+      st_shared_cluster_u32(peer_slot, static_cast<uint32_t>(t));
+      mbar_arrive_cluster(mapa_shared(smem_u32(&ring_full[slot]), 1));
+    }
+    mbar_arrive(smem_u32(&ring_full[slot]));
+    return true;
+  };
+  // Read the next tile index (all lanes of the calling warp, or one thread).
+  auto ring_take = [&](int slot, uint32_t rph, bool warp_wide, int& t) -> bool {
+    bool w = mbar_wait(smem_u32(&ring_full[slot]), rph, abort_flag, g0.timeout_ns);
+    if (warp_wide) w = __all_sync(0xffffffffu, w);
+    if (!w) return false;
+    if constexpr (kCG == 2) fence_acq_rel_cluster();  // the peer's copy is written remotely
+    t = *reinterpret_cast<volatile int*>(&tile_ring[slot]);
+    if (warp_wide) __syncwarp();
+    if (!warp_wide || lane == 0) {
+      const uint32_t e = smem_u32(&ring_empty[slot]);
+      if constexpr (kCG == 1)
+        mbar_arrive(e);
+      else
+        mbar_arrive_cluster(mapa_shared(e, 0));
+    }
+    return true;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer
+      // ---------------- TMA producer (every CTA loads its own halves)
+      if (g0.dep_wait == kDepBeforeLoads) griddep_wait();
       uint32_t stage = 0, phase = 0;
       uint32_t issued_mask = 0, issued_par = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        int mb, nb;
-        tile_coords(tile, g, mb, nb);
+      int rslot = 0;
+      uint32_t rph = 0;
+      for (int k = 0; ok; ++k) {
+        int tile;
+        if (leader) {
+          tile = (g0.tile_counter != nullptr) ? atomicAdd(g0.tile_counter, 1) : unit + k * n_units;
+          if (tile > num_tiles) tile = num_tiles;
+          ok = ring_publish(rslot, rph, tile);
+        } else {
+          ok = ring_take(rslot, rph, false, tile);
+        }
+        if (++rslot == kRing) {
+          rslot = 0;
+          rph ^= 1u;
+        }
+        if (!ok || tile >= num_tiles) break;
+        int prob, mb, nb;
+        locate(tile, prob, mb, nb);
+        const GemmArgs& g = prob ? g1 : g0;
+        const CUtensorMap* mA = prob ? &tmA1 : &tmA0;
+        const CUtensorMap* mB = prob ? &tmB1 : &tmB0;
+        const bool a_mn = prob ? kAMn1 : kAMn0;
+        const bool b_mn = prob ? kBMn1 : kBMn0;
+        const int m_cta = mb * Cfg::kUnitRows + static_cast<int>(rank) * BM;
+        const int n_cta = nb * BN + static_cast<int>(rank) * Cfg::kBRows;
         for (int kb = 0; kb < g.k_blocks; ++kb) {
-          if (!mbar_wait(smem_u32(&bar_empty[stage]), phase ^ 1u, abort_flag, g.timeout_ns)) {
+          if (!mbar_wait(smem_u32(&bar_empty[stage]), phase ^ 1u, abort_flag, g0.timeout_ns)) {
             ok = false;
             break;
           }
-          const uint32_t fb = smem_u32(&bar_full[stage]);
-          const uint32_t sa = smem_u32(smem + stage * kStageBytes);
+          const uint32_t fb_local = smem_u32(&bar_full[stage]);
+          uint32_t fb = fb_local;
+          if constexpr (kCG == 1) {
+            mbar_arrive_expect_tx(fb_local, Cfg::kStageBytes);
+          } else {
+            // the leader's barrier counts both CTAs' bytes
+            if (leader) mbar_arrive_expect_tx(fb_local, 2 * Cfg::kStageBytes);
+            fb = fb_local & kPairPeerBitMask;
+          }
+          const uint32_t sa = smem_u32(smem + stage * Cfg::kStageBytes);
           const uint32_t sb = sa + kABytes;
-          // An MN-major operand is loaded as 64-wide chunks along M/N.  A chunk
-          // that starts at or past the tensor's extent is not loaded at all:
-          // its shared-memory columns only feed output rows/columns that are
-          // never stored, and a box lying wholly outside the tensor is avoided.
-          uint32_t bytes = kStageBytes;
-          if (kAMn) {
+          if (a_mn) {
 #pragma unroll
             for (int c = 0; c < BM / 64; ++c)
-              if (mb * BM + c * 64 >= g.a_mn_extent) bytes -= 8192;
-          }
-          if (kBMn) {
-#pragma unroll
-            for (int c = 0; c < BN / 64; ++c)
-              if (nb * BN + c * 64 >= g.b_mn_extent) bytes -= 8192;
-          }
-          mbar_arrive_expect_tx(fb, bytes);
-          if (kAMn) {
-#pragma unroll
-            for (int c = 0; c < BM / 64; ++c)
-              if (mb * BM + c * 64 < g.a_mn_extent)
-                tma_load_2d(sa + c * 8192, &tmA, fb, mb * BM + c * 64, g.a_off + kb * BK);
+              load_2d<kCG>(sa + c * 8192, mA, fb, m_cta + c * 64, g.a_off + kb * BK);
           } else {
-            tma_load_2d(sa, &tmA, fb, kb * BK, g.a_off + mb * BM);
+            load_2d<kCG>(sa, mA, fb, kb * BK, g.a_off + m_cta);
           }
-          if (kBMn) {
+          if (b_mn) {
 #pragma unroll
-            for (int c = 0; c < BN / 64; ++c)
-              if (nb * BN + c * 64 < g.b_mn_extent)
-                tma_load_2d(sb + c * 8192, &tmB, fb, nb * BN + c * 64, g.b_off + kb * BK);
+            for (int c = 0; c < Cfg::kBRows / 64; ++c)
+              load_2d<kCG>(sb + c * 8192, mB, fb, n_cta + c * 64, g.b_off + kb * BK);
           } else {
-            tma_load_2d(sb, &tmB, fb, kb * BK, g.b_off + nb * BN);
+            load_2d<kCG>(sb, mB, fb, kb * BK, g.b_off + n_cta);
           }
           issued_mask |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -428,78 +552,118 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) {
-        record_timeout(g, abort_flag);
-        // Let every load already issued land before the CTA can exit.
-        for (int s = 0; s < kStages; ++s)
-          if ((issued_mask >> s) & 1u)
-            mbar_wait(smem_u32(&bar_full[s]), (issued_par >> s) & 1u, nullptr, g.timeout_ns);
+        record_timeout(g0, abort_flag);
+        // Let every load already issued land before the CTA can exit (the
+        // leader's full barriers also count the peer's bytes).
+        if (kCG == 1 || leader)
+          for (int s = 0; s < kStages; ++s)
+            if ((issued_mask >> s) & 1u)
+              mbar_wait(smem_u32(&bar_full[s]), (issued_par >> s) & 1u, nullptr, g0.timeout_ns);
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer
-      const uint32_t idesc = umma_idesc_bf16(BM, BN, kAMn, kBMn);
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (the pair's leader issues for both CTAs)
+      const uint32_t idesc0 = umma_idesc_bf16(BM * kCG, BN, kAMn0, kBMn0);
+      const uint32_t idesc1 = umma_idesc_bf16(BM * kCG, BN, kAMn1, kBMn1);
       uint32_t stage = 0, phase = 0;
       int it = 0;
       bool ok = true;
       bool issued = false;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+      int rslot = 0;
+      uint32_t rph = 0;
+      for (;; ++it) {
+        int tile;
+        ok = ring_take(rslot, rph, false, tile);
+        if (++rslot == kRing) {
+          rslot = 0;
+          rph ^= 1u;
+        }
+        if (!ok || tile >= num_tiles) break;
+        const int prob = (tile < tiles0) ? 0 : 1;
+        const int k_blocks = prob ? g1.k_blocks : g0.k_blocks;
+        const uint32_t idesc = prob ? idesc1 : idesc0;
+        const bool a_mn = prob ? kAMn1 : kAMn0;
+        const bool b_mn = prob ? kBMn1 : kBMn0;
         const uint32_t acc = it & 1;
         const uint32_t aph = (it >> 1) & 1;
-        if (!mbar_wait(smem_u32(&bar_tempty[acc]), aph ^ 1u, abort_flag, g.timeout_ns)) {
+        if (!mbar_wait(smem_u32(&bar_tempty[acc]), aph ^ 1u, abort_flag, g0.timeout_ns)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = 0; kb < g.k_blocks; ++kb) {
-          if (!mbar_wait(smem_u32(&bar_full[stage]), phase, abort_flag, g.timeout_ns)) {
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!mbar_wait(smem_u32(&bar_full[stage]), phase, abort_flag, g0.timeout_ns)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * kStageBytes);
+          const uint32_t sa = smem_u32(smem + stage * Cfg::kStageBytes);
           const uint32_t sb = sa + kABytes;
 #pragma unroll
           for (int j = 0; j < BK / 16; ++j) {
-            const uint64_t ad = kAMn ? umma_desc_sw128(sa + j * 2048, 8192, 1024)
+            const uint64_t ad = a_mn ? umma_desc_sw128(sa + j * 2048, 8192, 1024)
                                      : umma_desc_sw128(sa + j * 32, 16, 1024);
-            const uint64_t bd = kBMn ? umma_desc_sw128(sb + j * 2048, 8192, 1024)
+            const uint64_t bd = b_mn ? umma_desc_sw128(sb + j * 2048, 8192, 1024)
                                      : umma_desc_sw128(sb + j * 32, 16, 1024);
-            tc_mma_bf16(d_tmem, ad, bd, idesc, (kb > 0 || j > 0) ? 1u : 0u);
+            const uint32_t accum = (kb > 0 || j > 0) ? 1u : 0u;
+            if constexpr (kCG == 1)
+              tc_mma_bf16(d_tmem, ad, bd, idesc, accum);
+            else
+              tc_mma_bf16_pair(d_tmem, ad, bd, idesc, accum);
           }
           issued = true;
-          tc_commit(smem_u32(&bar_empty[stage]));
+          if constexpr (kCG == 1)
+            tc_commit(smem_u32(&bar_empty[stage]));
+          else
+            tc_commit_pair_mc(smem_u32(&bar_empty[stage]), 0x3);
           if (++stage == kStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(smem_u32(&bar_tfull[acc]));
+        if constexpr (kCG == 1)
+          tc_commit(smem_u32(&bar_tfull[acc]));
+        else
+          tc_commit_pair_mc(smem_u32(&bar_tfull[acc]), 0x3);
       }
       if (!ok) {
-        record_timeout(g, abort_flag);
+        record_timeout(g0, abort_flag);
         if (issued) {
           // Wait for the MMAs in flight before TMEM is released.
-          tc_commit(smem_u32(&bar_drain));
-          mbar_wait(smem_u32(&bar_drain), 0, nullptr, g.timeout_ns);
+          if constexpr (kCG == 1)
+            tc_commit(smem_u32(&bar_drain));
+          else
+            tc_commit_pair(smem_u32(&bar_drain));
+          mbar_wait(smem_u32(&bar_drain), 0, nullptr, g0.timeout_ns);
         }
       }
     }
   } else {
     // ---------------- epilogue warps
+    if (g0.dep_wait == kDepBeforeStores) griddep_wait();
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    uint8_t* stg = smem + kStages * kStageBytes + (warp - 2) * kStagingPerWarp;
+    uint8_t* stg = smem + kStages * Cfg::kStageBytes + (warp - 2) * kStagingPerWarp;
     int it = 0;
     int nstore = 0;  // TMA stores issued by this warp (selects the staging buffer)
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
-      int mb, nb;
-      tile_coords(tile, g, mb, nb);
+    int rslot = 0;
+    uint32_t rph = 0;
+    for (;; ++it) {
+      int tile;
+      ok = ring_take(rslot, rph, true, tile);
+      if (++rslot == kRing) {
+        rslot = 0;
+        rph ^= 1u;
+      }
+      if (!ok || tile >= num_tiles) break;
+      int prob, mb, nb;
+      locate(tile, prob, mb, nb);
       const uint32_t acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
-      bool w = mbar_wait(smem_u32(&bar_tfull[acc]), aph, abort_flag, g.timeout_ns);
+      bool w = mbar_wait(smem_u32(&bar_tfull[acc]), aph, abort_flag, g0.timeout_ns);
       w = __all_sync(0xffffffffu, w);
       if (!w) {
         ok = false;
@@ -507,18 +671,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const uint32_t taddr = tmem_base + acc * BN + (static_cast<uint32_t>(q * 32) << 16);
-      Epi::tile(ep, g, mb, nb, taddr, q, lane, stg, &tmOut, smem_u32(&bar_tempty[acc]), nstore);
+      const uint32_t tempty_local = smem_u32(&bar_tempty[acc]);
+      const uint32_t tempty = (kCG == 1) ? tempty_local : mapa_shared(tempty_local, 0);
+      const int m_base = mb * Cfg::kUnitRows + static_cast<int>(rank) * BM;
+      Epi::tile(prob ? ep1 : ep0, prob ? g1 : g0, m_base, nb, taddr, q, lane, stg,
+                prob ? &tmOut1 : &tmOut0, tempty, nstore);
     }
     if (lane == 0) {
       bulk_wait_group_all();
-      if (!ok) record_timeout(g, abort_flag);
+      if (!ok) record_timeout(g0, abort_flag);
     }
   }
 
   __syncthreads();
+  if constexpr (kCG == 2) cluster_sync();  // neither CTA leaves while its peer may still use it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if constexpr (kCG == 1)
+      tmem_dealloc(tmem_base, kTmemCols);
+    else
+      tmem_dealloc_pair(tmem_base, kTmemCols);
   }
 }
 
