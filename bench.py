@@ -180,6 +180,23 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- ranks
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest value of `x` over all ranks (the slowest rank's time)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, units_per_rank_step: int, steps: int, ms: float) -> float:
+    """Units all ranks processed per second, timed by the slowest rank."""
+    return world * units_per_rank_step * steps / (ms / 1e3)
+
+
 # ---------------------------------------------------------------- own arm
 def source_digest():
     h = hashlib.sha256()
@@ -274,12 +291,9 @@ def run_own(args, rank, world, local_rank):
     clocks = sampler.stop()
     ms = e0.elapsed_time(e1)
     barrier()
-    if world > 1:
-        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms, world, dev)
     ms_step = ms / args.steps
-    value = world * N * args.steps / (ms / 1e3)
+    value = whole_job_rate(world, N, args.steps, ms)
 
     # ---- per-kernel accounting: the same K steps again, with a CUDA event pair
     # recorded by the library around every kernel it launches (on this stream)
@@ -320,11 +334,8 @@ def run_own(args, rank, world, local_rank):
     torch.cuda.synchronize()
     ms_e2e = e0.elapsed_time(e1)
     barrier()
-    if world > 1:
-        tt = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_e2e = float(tt.item())
-    e2e_value = world * N * e2e_steps / (ms_e2e / 1e3)
+    ms_e2e = max_over_ranks(ms_e2e, world, dev)
+    e2e_value = whole_job_rate(world, N, e2e_steps, ms_e2e)
     h2d = h_host.numel() * 2 + y_host.numel() * 8
     d2h = 4 + 8
 

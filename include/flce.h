@@ -154,6 +154,15 @@ flce_status flce_forward_noalloc(const void* hidden, const void* weight, const i
  * the workspace since the last flce_forward (FLCE_OK if none). */
 flce_status flce_get_status(const void* workspace, void* stream);
 
+/* Self-test of failure reporting: launches one tiny kernel whose thread waits
+ * on an mbarrier that nothing arrives on, through the same bounded wait the
+ * GEMM pipelines use, with a limit of timeout_ms (1..10000).  The wait runs
+ * out, the kernel records the timeout bit in the workspace status word and
+ * returns, so the following flce_get_status() reports FLCE_ERR_TIMEOUT and the
+ * CUDA context stays usable.  No fault, trap or hang is involved; the next
+ * flce_forward clears the status.  (Test hook; no counterpart on the pages.) */
+flce_status flce_selftest_wait_timeout(void* workspace, int32_t timeout_ms, void* stream);
+
 /* Human-readable name of a status code (static storage). */
 const char* flce_status_string(int32_t status);
 

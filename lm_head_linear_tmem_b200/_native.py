@@ -37,6 +37,7 @@ SIGNATURES = {
     "flce_forward_noalloc": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32,
                                      c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "flce_get_status": (c_i32, [c_vp, c_vp]),
+    "flce_selftest_wait_timeout": (c_i32, [c_vp, c_i32, c_vp]),
     "flce_status_string": (ctypes.c_char_p, [c_i32]),
     "flce_version": (c_i32, []),
     "flce_launch_count": (c_u64, []),

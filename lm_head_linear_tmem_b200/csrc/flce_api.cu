@@ -699,6 +699,20 @@ flce_status flce_get_status(const void* workspace, void* stream) {
   return FLCE_OK;
 }
 
+flce_status flce_selftest_wait_timeout(void* workspace, int32_t timeout_ms, void* stream) {
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return FLCE_ERR_ARG;
+  if (timeout_ms < 1 || timeout_ms > 10000) return FLCE_ERR_ARG;
+  DevInfo* d = nullptr;
+  flce_status s = device_info(&d);
+  if (s != FLCE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned int* status = ws_status(workspace);
+  const unsigned long long ns = static_cast<unsigned long long>(timeout_ms) * 1000000ull;
+  const cudaError_t e = launch(kHelper, st, [&] { selftest_wait_kernel<<<1, 32, 0, st>>>(status, ns); });
+  return e == cudaSuccess ? FLCE_OK : cuda_fail(e);
+}
+
 const char* flce_status_string(int32_t status) {
   switch (status) {
     case FLCE_OK: return "FLCE_OK";

@@ -149,6 +149,17 @@ __global__ void __launch_bounds__(kFinalThreads)
   if (t == 0) *n_valid_out = sc[0];
 }
 
+// Waits, bounded, on an mbarrier that nothing completes; records the timeout
+// in the status word (the same wait and report as the GEMM pipelines).
+__global__ void selftest_wait_kernel(unsigned int* status, unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+    if (!mbar_wait(smem_u32(&bar), 0, nullptr, timeout_ns)) atomicOr(status, kStatusTimeout);
+  }
+}
+
 // ------------------------------------------------------------------ fp32 path
 constexpr int kSimtThreads = 256;
 constexpr int kSimtChunk = 1024;
