@@ -344,10 +344,17 @@ def run_own(args, rank, world, local_rank):
 
     peaks, peak_src = load_peaks()
     flops_step = w.flops_per_step
+    # Work the kernels execute: the forward covers every row; the backward GEMMs
+    # cover the non-ignored rows only (rows with ignore_index have exactly zero
+    # gradient and are compacted away) unless FLCE_BWD_COMPACT=0.
+    n_valid = int((inp.labels != fi.IGNORE_INDEX).sum())
+    compact = os.environ.get("FLCE_BWD_COMPACT", "1") != "0"
+    n_bwd = n_valid if compact else N
+    executed_step = 2.0 * N * H * V + 6.0 * n_bwd * H * V
     # the dominant kernel (largest device time) and its roofline
     # FLOP per step of each kernel kind (summed over its launches)
-    credited = {"fwd_gemm_softmax_stats": 2.0 * N * H * V, "bwd_dz_gemm": 2.0 * N * H * V,
-                "bwd_dhidden_dweight_gemm": 4.0 * N * H * V}
+    credited = {"fwd_gemm_softmax_stats": 2.0 * N * H * V, "bwd_dz_gemm": 2.0 * n_bwd * H * V,
+                "bwd_dhidden_dweight_gemm": 4.0 * n_bwd * H * V}
     dom = max(kinds, key=lambda k: kinds[k]["ms_total"]) if kinds else None
     roofline = None
     if dom in credited:
@@ -379,6 +386,11 @@ def run_own(args, rank, world, local_rank):
                    "l2": "inputs larger than L2 (weight 1 GiB bf16), no flush"},
         "tensor_peak_pct": {"credited_tflops": tflops, "flops_per_step": flops_step,
                             "frac_of_burst": tflops / burst, "frac_of_sustained": tflops / sust,
+                            "executed_flops_per_step": executed_step,
+                            "executed_tflops": executed_step / (ms_step / 1e3) / 1e12,
+                            "executed_frac_of_sustained":
+                                executed_step / (ms_step / 1e3) / 1e12 / sust,
+                            "backward_rows": n_bwd, "tokens": N,
                             "peak_source": peak_src},
         "roofline": roofline,
         "kernels": kinds,

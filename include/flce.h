@@ -102,19 +102,28 @@ flce_status flce_forward(const void* hidden, const void* weight, const int64_t* 
                          int32_t reduction, int32_t dtype, float* loss, int64_t* num_tokens,
                          float* lse, void* workspace, size_t workspace_bytes, void* stream);
 
+/* flce_backward flags. */
+#define FLCE_ACCUMULATE_DHIDDEN 1 /* d_hidden += gradient (else overwritten) */
+#define FLCE_ACCUMULATE_DWEIGHT 2 /* d_weight += gradient (else overwritten) */
+
 /* Backward of the loss returned by flce_forward with the same arguments.
  *   lse          device float[N]  from flce_forward
  *   grad_output  device float[1]  upstream gradient of the loss; NULL means 1.0
  *   grad_scale   host float       extra factor (micro-batch / token weighting)
  *   num_valid    device int64[1]  n (the true count, also for 'mean');
  *                                 NULL: the library counts it on the device
- *   d_hidden     device float[N*H]  overwritten
- *   d_weight     device float[V*H]  overwritten */
+ *   d_hidden     device float[N*H]  overwritten, or accumulated into
+ *   d_weight     device float[V*H]  overwritten, or accumulated into
+ *   flags        FLCE_ACCUMULATE_DHIDDEN | FLCE_ACCUMULATE_DWEIGHT, or 0.
+ * Accumulating into d_weight across the micro-batches of one optimizer step
+ * (each with grad_scale = 1 / the step's total non-ignored count) gives the
+ * token-weighted gradient of the whole batch (modelscope/twinkle PR #335,
+ * item 2). */
 flce_status flce_backward(const void* hidden, const void* weight, const int64_t* labels,
                           const float* lse, int64_t N, int64_t H, int64_t V,
                           int64_t ignore_index, float softcap, int32_t reduction, int32_t dtype,
                           const float* grad_output, float grad_scale, const int64_t* num_valid,
-                          float* d_hidden, float* d_weight, void* workspace,
+                          float* d_hidden, float* d_weight, int32_t flags, void* workspace,
                           size_t workspace_bytes, void* stream);
 
 /* Size of the library-owned device buffer behind flce_forward_noalloc. */

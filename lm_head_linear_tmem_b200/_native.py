@@ -25,6 +25,7 @@ STATUS_NAMES = {
 }
 SUM, MEAN = 0, 1
 BF16, FP32 = 0, 1
+ACCUMULATE_DHIDDEN, ACCUMULATE_DWEIGHT = 1, 2
 
 # Every symbol include/flce.h declares, with its ctypes signature.
 SIGNATURES = {
@@ -32,7 +33,7 @@ SIGNATURES = {
     "flce_forward": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32, c_i32,
                              c_i32, c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),
     "flce_backward": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32,
-                              c_i32, c_i32, c_vp, c_f32, c_vp, c_vp, c_vp, c_vp, c_size,
+                              c_i32, c_i32, c_vp, c_f32, c_vp, c_vp, c_vp, c_i32, c_vp, c_size,
                               c_vp]),
     "flce_forward_noalloc": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32,
                                      c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp]),

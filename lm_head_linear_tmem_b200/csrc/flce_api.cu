@@ -192,20 +192,45 @@ int64_t bwd_launches(int64_t N, int64_t V) {
   return 3 * ((N + c.tc - 1) / c.tc) * ((V + c.vc - 1) / c.vc);
 }
 
-// Backward workspace: header | tile counters | dZ block (1024-aligned).
-size_t bwd_counters_offset() { return kHeaderBytes; }
-size_t bwd_gblock_offset(int64_t N, int64_t V) {
-  return align_up(kHeaderBytes + 4 * static_cast<size_t>(bwd_launches(N, V)), 1024);
-}
+// Backward workspace: header | tile counters | row compaction (permutation,
+// compact labels and lse, per-block counts, valid count) | compact hidden
+// [N, H] bf16 | dZ block.
+struct BwdLayout {
+  size_t counters, perm, labels_c, lse_c, block_valid, n_valid_c, hidden_c, gblock, end;
+};
 
-size_t bwd_bytes(int64_t N, int64_t V, bool bf16) {
-  if (!bf16) return kHeaderBytes;
+BwdLayout bwd_layout(int64_t N, int64_t H, int64_t V) {
+  BwdLayout L{};
   const Chunking c = chunking(N, V);
-  return bwd_gblock_offset(N, V) + static_cast<size_t>(c.tc) * c.vc * 2 + 1024;
+  const size_t nblk = static_cast<size_t>((N + kCompactThreads - 1) / kCompactThreads);
+  size_t off = kHeaderBytes;
+  L.counters = off;
+  off = align_up(off + 4 * static_cast<size_t>(bwd_launches(N, V)), 256);
+  L.perm = off;
+  off = align_up(off + 4 * static_cast<size_t>(N), 256);
+  L.labels_c = off;
+  off = align_up(off + 8 * static_cast<size_t>(N), 256);
+  L.lse_c = off;
+  off = align_up(off + 4 * static_cast<size_t>(N), 256);
+  L.block_valid = off;
+  off = align_up(off + 4 * nblk, 256);
+  L.n_valid_c = off;
+  off = align_up(off + 8, 1024);
+  L.hidden_c = off;
+  off = align_up(off + 2 * static_cast<size_t>(N) * static_cast<size_t>(H), 1024);
+  L.gblock = off;
+  off += static_cast<size_t>(c.tc) * c.vc * 2 + 1024;
+  L.end = off;
+  return L;
 }
 
-size_t ws_bytes(int64_t N, int64_t V, bool bf16) {
-  return align_up(std::max(fwd_layout(N, V, bf16).end, bwd_bytes(N, V, bf16)), 256);
+size_t bwd_bytes(int64_t N, int64_t H, int64_t V, bool bf16) {
+  if (!bf16) return kHeaderBytes;
+  return bwd_layout(N, H, V).end;
+}
+
+size_t ws_bytes(int64_t N, int64_t H, int64_t V, bool bf16) {
+  return align_up(std::max(fwd_layout(N, V, bf16).end, bwd_bytes(N, H, V, bf16)), 256);
 }
 
 unsigned int* ws_status(void* ws) { return reinterpret_cast<unsigned int*>(ws); }
@@ -219,6 +244,14 @@ long long* ws_nvalid(void* ws) {
 int cta_group() {
   const char* s = std::getenv("FLCE_CTA_GROUP");
   return (s != nullptr && std::atoi(s) == 1) ? 1 : 2;
+}
+
+// Backward row compaction: token rows whose label is ignore_index are left out
+// of the backward GEMMs (default), or FLCE_BWD_COMPACT=0 keeps every row
+// (read at every call).
+bool bwd_compact() {
+  const char* s = std::getenv("FLCE_BWD_COMPACT");
+  return !(s != nullptr && std::atoi(s) == 0);
 }
 
 // Backward chunk schedule: the dHidden and dWeight GEMMs of a chunk share one
@@ -257,7 +290,7 @@ flce_status check_common(const void* hidden, const void* weight, const int64_t* 
   if (!aligned16(hidden) || !aligned16(weight) || !aligned16(ws)) return FLCE_ERR_ARG;
   if ((reinterpret_cast<uintptr_t>(labels) & 7u) != 0) return FLCE_ERR_ARG;
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return FLCE_ERR_ARG;
-  if (ws_size < ws_bytes(N, V, dtype == FLCE_BF16)) return FLCE_ERR_WORKSPACE;
+  if (ws_size < ws_bytes(N, H, V, dtype == FLCE_BF16)) return FLCE_ERR_WORKSPACE;
   return FLCE_OK;
 }
 
@@ -465,20 +498,69 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
                           const int64_t* labels, const float* lse, int64_t N, int64_t H,
                           int64_t V, int64_t ignore_index, float softcap, int32_t reduction,
                           const float* grad_output, float grad_scale, const long long* n_valid,
-                          float* d_hidden, float* d_weight, void* ws, cudaStream_t st) {
+                          bool n_valid_is_count, float* d_hidden, float* d_weight,
+                          int32_t flags, void* ws, cudaStream_t st) {
+  const bool acc_dh = (flags & FLCE_ACCUMULATE_DHIDDEN) != 0;
+  const bool acc_dw = (flags & FLCE_ACCUMULATE_DWEIGHT) != 0;
   const Chunking ck = chunking(N, V);
+  const BwdLayout BL = bwd_layout(N, H, V);
   char* w = static_cast<char*>(ws);
-  void* gbuf = w + bwd_gblock_offset(N, V);
-  int* counters = reinterpret_cast<int*>(w + bwd_counters_offset());
+  void* gbuf = w + BL.gblock;
+  int* counters = reinterpret_cast<int*>(w + BL.counters);
   int next_counter = 0;
   {
     const cudaError_t e = cudaMemsetAsync(counters, 0, 4 * bwd_launches(N, V), st);
     if (e != cudaSuccess) return cuda_fail(e);
   }
 
+  // Row compaction: the GEMMs see the valid token rows first (compact hidden,
+  // labels and lse), the device-side count bounds their token-row dimension,
+  // and dHidden rows are scattered back through the permutation.
+  const bool compact = bwd_compact();
+  const void* hid = hidden;
+  const int64_t* lab = labels;
+  const float* lsev = lse;
+  int* perm = nullptr;
+  const long long* rows_valid = nullptr;
+  if (compact) {
+    perm = reinterpret_cast<int*>(w + BL.perm);
+    int64_t* labels_c = reinterpret_cast<int64_t*>(w + BL.labels_c);
+    float* lse_c = reinterpret_cast<float*>(w + BL.lse_c);
+    int* block_valid = reinterpret_cast<int*>(w + BL.block_valid);
+    long long* n_valid_c = reinterpret_cast<long long*>(w + BL.n_valid_c);
+    void* hidden_c = w + BL.hidden_c;
+    const int n = static_cast<int>(N);
+    const int nblk = (n + kCompactThreads - 1) / kCompactThreads;
+    cudaError_t e = launch(kHelper, st, [&] {
+      compact_count_kernel<<<nblk, kCompactThreads, 0, st>>>(labels, n, ignore_index, block_valid);
+    });
+    if (e == cudaSuccess)
+      e = launch(kHelper, st, [&] {
+        compact_scan_kernel<<<1, kCompactThreads, 0, st>>>(block_valid, nblk, n_valid_c);
+      });
+    if (e == cudaSuccess)
+      e = launch(kHelper, st, [&] {
+        compact_scatter_kernel<<<nblk, kCompactThreads, 0, st>>>(
+            labels, lse, n, ignore_index, block_valid, n_valid_c, perm, labels_c, lse_c);
+      });
+    if (e == cudaSuccess)
+      e = launch(kHelper, st, [&] {
+        gather_rows_kernel<<<n, 256, 0, st>>>(
+            static_cast<const uint4*>(hidden), static_cast<int>(H / 8), n, perm, n_valid_c,
+            static_cast<uint4*>(hidden_c), reinterpret_cast<float4*>(d_hidden),
+            static_cast<int>(H / 4), acc_dh ? 0 : 1);
+      });
+    if (e != cudaSuccess) return cuda_fail(e);
+    hid = hidden_c;
+    lab = labels_c;
+    lsev = lse_c;
+    rows_valid = n_valid_c;
+    if (n_valid_is_count) n_valid = n_valid_c;  // the library's own count serves both
+  }
+
   CUtensorMap t_hid_k, t_hid_mn, t_w_k, t_w_mn, t_dh, t_dw;
-  if (!make_map(&t_hid_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hidden, H, N, H * 2, BK, BM) ||
-      !make_map(&t_hid_mn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hidden, H, N, H * 2, 64, BK) ||
+  if (!make_map(&t_hid_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hid, H, N, H * 2, BK, BM) ||
+      !make_map(&t_hid_mn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hid, H, N, H * 2, 64, BK) ||
       !make_map(&t_w_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, weight, H, V, H * 2, BK, b_box_rows()) ||
       !make_map(&t_w_mn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, weight, H, V, H * 2, 64, BK) ||
       !make_map(&t_dh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d_hidden, H, N, H * 4, 32, 32) ||
@@ -514,17 +596,21 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
       gz.status = ws_status(ws);
       gz.timeout_ns = tmo;
       gz.tile_counter = counters + next_counter++;
+      gz.rows_valid = rows_valid;
+      gz.rows_base = static_cast<int>(t0);
+      gz.rows_host = rows;
+      gz.rows_dim = kRowsM;
       // dZ overwrites the block the previous chunk's dHidden/dWeight GEMMs read:
       // its main loop may start early, its first store waits for them
       gz.dep_wait = (t0 > 0 || v0 > 0) ? kDepBeforeStores : kDepNone;
       cudaError_t e;
       const GemmProblem pz{&t_hid_k, &t_w_k, &t_g_store, rows, gz};
       if (softcap > 0.f) {
-        DzEpi<true>::Params ep{labels, lse, ignore_index, static_cast<int>(t0), rows,
+        DzEpi<true>::Params ep{lab, lsev, ignore_index, static_cast<int>(t0), rows,
                                static_cast<int>(v0), cols, softcap, 1.0f / softcap};
         e = run_gemm<DzEpi<true>, false, false>(d, kSlotDzCap, kBwdDz, pz, ep, nullptr, ep, st);
       } else {
-        DzEpi<false>::Params ep{labels, lse, ignore_index, static_cast<int>(t0), rows,
+        DzEpi<false>::Params ep{lab, lsev, ignore_index, static_cast<int>(t0), rows,
                                 static_cast<int>(v0), cols, 0.f, 0.f};
         e = run_gemm<DzEpi<false>, false, false>(d, kSlotDz, kBwdDz, pz, ep, nullptr, ep, st);
       }
@@ -540,9 +626,14 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
       gh.status = ws_status(ws);
       gh.timeout_ns = tmo;
       gh.tile_counter = counters + next_counter++;
+      gh.rows_valid = rows_valid;
+      gh.rows_base = static_cast<int>(t0);
+      gh.rows_host = rows;
+      gh.rows_dim = kRowsM;
       gh.dep_wait = kDepBeforeLoads;  // reads the dZ block written just before
-      StoreEpi::Params eh{static_cast<int>(t0), v0 > 0 ? 1 : 0, static_cast<int>(H),
-                          static_cast<int>(N), grad_output, grad_scale, n_valid, mean};
+      StoreEpi::Params eh{static_cast<int>(t0), (v0 > 0 || acc_dh) ? 1 : 0, static_cast<int>(H),
+                          static_cast<int>(N), grad_output, grad_scale, n_valid, mean,
+                          perm, rows_valid, d_hidden, static_cast<int>(H)};
 
       // 3) dWeight[v0:v0+cols] (+)= dZ^T . hidden[t0:t0+rows]
       GemmArgs gw{};
@@ -554,9 +645,15 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
       gw.status = ws_status(ws);
       gw.timeout_ns = tmo;
       gw.tile_counter = counters + next_counter++;
+      gw.rows_valid = rows_valid;
+      gw.rows_base = static_cast<int>(t0);
+      gw.rows_host = rows;
+      gw.rows_dim = kRowsK;
+      gw.zero_if_empty = (t0 == 0 && !acc_dw) ? 1 : 0;  // the first chunk overwrites dWeight
       gw.dep_wait = kDepBeforeLoads;
-      StoreEpi::Params ew{static_cast<int>(v0), t0 > 0 ? 1 : 0, static_cast<int>(H),
-                          static_cast<int>(V), grad_output, grad_scale, n_valid, mean};
+      StoreEpi::Params ew{static_cast<int>(v0), (t0 > 0 || acc_dw) ? 1 : 0, static_cast<int>(H),
+                          static_cast<int>(V), grad_output, grad_scale, n_valid, mean,
+                          nullptr, nullptr, nullptr, 0};
 
       const GemmProblem ph{&t_g_k, &t_w_mn, &t_dh, rows, gh};
       const GemmProblem pw{&t_g_mn, &t_hid_mn, &t_dw, cols, gw};
@@ -578,7 +675,9 @@ flce_status backward_fp32(DevInfo* d, const void* hidden, const void* weight,
                           const int64_t* labels, const float* lse, int64_t N, int64_t H,
                           int64_t V, int64_t ignore_index, float softcap, int32_t reduction,
                           const float* grad_output, float grad_scale, const long long* n_valid,
-                          float* d_hidden, float* d_weight, cudaStream_t st) {
+                          float* d_hidden, float* d_weight, int32_t flags, cudaStream_t st) {
+  const int acc_dh = (flags & FLCE_ACCUMULATE_DHIDDEN) ? 1 : 0;
+  const int acc_dw = (flags & FLCE_ACCUMULATE_DWEIGHT) ? 1 : 0;
   const int n = static_cast<int>(N), h = static_cast<int>(H), v = static_cast<int>(V);
   const int mean = reduction == FLCE_MEAN;
   const size_t sh_dh = (2 * static_cast<size_t>(h) + kSimtChunk) * sizeof(float);
@@ -591,14 +690,14 @@ flce_status backward_fp32(DevInfo* d, const void* hidden, const void* weight,
     e = launch(kSimt, st, [&] {
       simt_dh_kernel<<<n, kSimtThreads, sh_dh, st>>>(
           static_cast<const float*>(hidden), static_cast<const float*>(weight), labels, lse, n, h,
-          v, ignore_index, softcap, grad_output, grad_scale, n_valid, mean, d_hidden);
+          v, ignore_index, softcap, grad_output, grad_scale, n_valid, mean, acc_dh, d_hidden);
     });
     if (e != cudaSuccess) return cuda_fail(e);
   }
   e = launch(kSimt, st, [&] {
     simt_dw_kernel<<<v, kSimtThreads, sh_dw, st>>>(
         static_cast<const float*>(hidden), static_cast<const float*>(weight), labels, lse, n, h, v,
-        ignore_index, softcap, grad_output, grad_scale, n_valid, mean, d_weight);
+        ignore_index, softcap, grad_output, grad_scale, n_valid, mean, acc_dw, d_weight);
   });
   if (e != cudaSuccess) return cuda_fail(e);
   return FLCE_OK;
@@ -614,7 +713,7 @@ extern "C" {
 size_t flce_workspace_bytes(int64_t N, int64_t H, int64_t V, int32_t dtype) {
   if (N < 0 || V < 1 || H < 8 || N > kMaxDim || V > kMaxDim) return 0;
   if (dtype != FLCE_BF16 && dtype != FLCE_FP32) return 0;
-  return ws_bytes(N, V, dtype == FLCE_BF16);
+  return ws_bytes(N, H, V, dtype == FLCE_BF16);
 }
 
 flce_status flce_forward(const void* hidden, const void* weight, const int64_t* labels,
@@ -649,8 +748,9 @@ flce_status flce_backward(const void* hidden, const void* weight, const int64_t*
                           const float* lse, int64_t N, int64_t H, int64_t V,
                           int64_t ignore_index, float softcap, int32_t reduction, int32_t dtype,
                           const float* grad_output, float grad_scale, const int64_t* num_valid,
-                          float* d_hidden, float* d_weight, void* workspace,
+                          float* d_hidden, float* d_weight, int32_t flags, void* workspace,
                           size_t workspace_bytes, void* stream) {
+  if ((flags & ~(FLCE_ACCUMULATE_DHIDDEN | FLCE_ACCUMULATE_DWEIGHT)) != 0) return FLCE_ERR_ARG;
   flce_status s = check_common(hidden, weight, labels, N, H, V, softcap, reduction, dtype,
                                workspace, workspace_bytes);
   if (s != FLCE_OK) return s;
@@ -665,11 +765,13 @@ flce_status flce_backward(const void* hidden, const void* weight, const int64_t*
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (N == 0) {
+    if (flags & FLCE_ACCUMULATE_DWEIGHT) return FLCE_OK;  // adds nothing
     e = cudaMemsetAsync(d_weight, 0, static_cast<size_t>(V) * H * sizeof(float), st);
     return e == cudaSuccess ? FLCE_OK : cuda_fail(e);
   }
   const long long* nv = reinterpret_cast<const long long*>(num_valid);
-  if (nv == nullptr) {
+  const bool own_count = (nv == nullptr);
+  if (nv == nullptr && !(dtype == FLCE_BF16 && bwd_compact())) {
     long long* out = ws_nvalid(workspace);
     e = launch(kHelper, st, [&] {
       count_valid_kernel<<<1, kFinalThreads, 0, st>>>(labels, static_cast<int>(N), ignore_index,
@@ -680,10 +782,10 @@ flce_status flce_backward(const void* hidden, const void* weight, const int64_t*
   }
   if (dtype == FLCE_BF16)
     return backward_bf16(d, hidden, weight, labels, lse, N, H, V, ignore_index, softcap,
-                         reduction, grad_output, grad_scale, nv, d_hidden, d_weight, workspace,
-                         st);
+                         reduction, grad_output, grad_scale, nv, own_count, d_hidden, d_weight,
+                         flags, workspace, st);
   return backward_fp32(d, hidden, weight, labels, lse, N, H, V, ignore_index, softcap, reduction,
-                       grad_output, grad_scale, nv, d_hidden, d_weight, st);
+                       grad_output, grad_scale, nv, d_hidden, d_weight, flags, st);
 }
 
 flce_status flce_get_status(const void* workspace, void* stream) {

@@ -149,6 +149,110 @@ __global__ void __launch_bounds__(kFinalThreads)
   if (t == 0) *n_valid_out = sc[0];
 }
 
+// ------------------------------------------------------------------ row compaction
+// The backward skips token rows whose label is ignore_index (their gradient is
+// exactly zero).  A stable compaction puts the valid rows first, in order, then
+// the ignored rows, in order: perm[j] is the original row of compact row j.
+constexpr int kCompactThreads = 1024;
+
+// Valid rows per block of kCompactThreads rows.
+__global__ void __launch_bounds__(kCompactThreads)
+    compact_count_kernel(const int64_t* __restrict__ labels, int N, int64_t ignore_index,
+                         int* __restrict__ block_valid) {
+  __shared__ int warp_sum[kCompactThreads / 32];
+  const int i = blockIdx.x * kCompactThreads + threadIdx.x;
+  const bool v = (i < N) && (labels[i] != ignore_index);
+  const unsigned m = __ballot_sync(0xffffffffu, v);
+  if ((threadIdx.x & 31) == 0) warp_sum[threadIdx.x >> 5] = __popc(m);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int s = 0;
+    for (int w = 0; w < kCompactThreads / 32; ++w) s += warp_sum[w];
+    block_valid[blockIdx.x] = s;
+  }
+}
+
+// One block: exclusive prefix sum of the per-block counts (in place) and the
+// total number of valid rows.
+__global__ void __launch_bounds__(kCompactThreads)
+    compact_scan_kernel(int* __restrict__ block_valid, int nblk, long long* __restrict__ n_valid) {
+  __shared__ int carry;
+  __shared__ int warp_sum[kCompactThreads / 32];
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int base = 0; base < nblk; base += kCompactThreads) {
+    const int b = base + threadIdx.x;
+    const int x = (b < nblk) ? block_valid[b] : 0;
+    int incl = x;  // inclusive scan within the warp
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
+    __syncthreads();
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += warp_sum[w];
+    const int excl = carry + before + incl - x;
+    __syncthreads();
+    if (b < nblk) block_valid[b] = excl;
+    if (threadIdx.x == kCompactThreads - 1) carry = excl + x;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *n_valid = carry;
+}
+
+// perm[j], and the compact labels and lse of every compact row: valid rows keep
+// theirs; ignored rows get ignore_index and lse 0.
+__global__ void __launch_bounds__(kCompactThreads)
+    compact_scatter_kernel(const int64_t* __restrict__ labels, const float* __restrict__ lse,
+                           int N, int64_t ignore_index, const int* __restrict__ block_offset,
+                           const long long* __restrict__ n_valid, int* __restrict__ perm,
+                           int64_t* __restrict__ labels_c, float* __restrict__ lse_c) {
+  __shared__ int warp_sum[kCompactThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int i = blockIdx.x * kCompactThreads + threadIdx.x;
+  const int64_t y = (i < N) ? labels[i] : ignore_index;
+  const bool v = (i < N) && (y != ignore_index);
+  const unsigned m = __ballot_sync(0xffffffffu, v);
+  if (lane == 0) warp_sum[warp] = __popc(m);
+  __syncthreads();
+  int before = 0;
+  for (int w = 0; w < warp; ++w) before += warp_sum[w];
+  const int rank_v = block_offset[blockIdx.x] + before + __popc(m & ((1u << lane) - 1u));
+  if (i < N) {
+    const int j = v ? rank_v : static_cast<int>(*n_valid) + (i - rank_v);
+    perm[j] = i;
+    labels_c[j] = v ? y : ignore_index;
+    lse_c[j] = v ? lse[i] : 0.f;
+  }
+}
+
+// Compact hidden: row j < n_valid is hidden[perm[j]]; rows past n_valid are
+// zero.  Ignored rows of d_hidden are zeroed here (unless accumulating).
+__global__ void __launch_bounds__(256)
+    gather_rows_kernel(const uint4* __restrict__ hidden, int H16, int N,
+                       const int* __restrict__ perm, const long long* __restrict__ n_valid,
+                       uint4* __restrict__ hidden_c, float4* __restrict__ d_hidden, int H4,
+                       int zero_ignored_dh) {
+  const int j = blockIdx.x;
+  if (j >= N) return;
+  const long long nv = *n_valid;
+  uint4* dst = hidden_c + static_cast<size_t>(j) * H16;
+  if (j < nv) {
+    const uint4* src = hidden + static_cast<size_t>(perm[j]) * H16;
+    for (int k = threadIdx.x; k < H16; k += blockDim.x) dst[k] = src[k];
+  } else {
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    for (int k = threadIdx.x; k < H16; k += blockDim.x) dst[k] = z;
+    if (zero_ignored_dh) {
+      float4* o = d_hidden + static_cast<size_t>(perm[j]) * H4;
+      const float4 zf = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int k = threadIdx.x; k < H4; k += blockDim.x) o[k] = zf;
+    }
+  }
+}
+
 // Waits, bounded, on an mbarrier that nothing completes; records the timeout
 // in the status word (the same wait and report as the GEMM pipelines).
 __global__ void selftest_wait_kernel(unsigned int* status, unsigned long long timeout_ns) {
@@ -234,7 +338,7 @@ __global__ void __launch_bounds__(kSimtThreads)
     simt_dh_kernel(const float* __restrict__ hidden, const float* __restrict__ weight,
                    const int64_t* __restrict__ labels, const float* __restrict__ lse, int N,
                    int H, int V, int64_t ignore_index, float softcap, const float* grad_output,
-                   float grad_scale, const long long* n_valid, int mean,
+                   float grad_scale, const long long* n_valid, int mean, int accumulate,
                    float* __restrict__ d_hidden) {
   extern __shared__ float sh[];
   float* h = sh;
@@ -278,7 +382,10 @@ __global__ void __launch_bounds__(kSimtThreads)
     }
     __syncthreads();
   }
-  for (int k = t; k < H; k += kSimtThreads) d_hidden[static_cast<size_t>(row) * H + k] = acc[k];
+  for (int k = t; k < H; k += kSimtThreads) {
+    float* o = d_hidden + static_cast<size_t>(row) * H + k;
+    *o = accumulate ? *o + acc[k] : acc[k];
+  }
 }
 
 // One block per vocab row: dWeight[v] = sum_i dZ[i, v] hidden[i].
@@ -287,7 +394,7 @@ __global__ void __launch_bounds__(kSimtThreads)
     simt_dw_kernel(const float* __restrict__ hidden, const float* __restrict__ weight,
                    const int64_t* __restrict__ labels, const float* __restrict__ lse, int N,
                    int H, int V, int64_t ignore_index, float softcap, const float* grad_output,
-                   float grad_scale, const long long* n_valid, int mean,
+                   float grad_scale, const long long* n_valid, int mean, int accumulate,
                    float* __restrict__ d_weight) {
   extern __shared__ float sh[];
   float* w = sh;
@@ -329,7 +436,10 @@ __global__ void __launch_bounds__(kSimtThreads)
     }
     __syncthreads();
   }
-  for (int k = t; k < H; k += kSimtThreads) d_weight[static_cast<size_t>(v) * H + k] = acc[k];
+  for (int k = t; k < H; k += kSimtThreads) {
+    float* o = d_weight + static_cast<size_t>(v) * H + k;
+    *o = accumulate ? *o + acc[k] : acc[k];
+  }
 }
 
 }  // namespace flce

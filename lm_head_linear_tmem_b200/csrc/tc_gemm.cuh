@@ -84,7 +84,21 @@ struct GemmArgs {
   int dep_wait;       // what waits for the previous kernel on the stream (launched
                       // as a programmatic dependent): kDepNone, kDepBeforeLoads
                       // (operands it produced), kDepBeforeStores (an output it reads)
+  // Token rows bounded on the device: when rows_valid is set, only the first
+  // clamp(*rows_valid - rows_base, 0, rows_host) token rows of this launch are
+  // worked on.  rows_dim says which GEMM dimension they are (kRowsM, kRowsK);
+  // with kRowsK an empty range drops the tiles, or (zero_if_empty) makes them
+  // write zeros.
+  const long long* rows_valid;
+  int rows_base;
+  int rows_host;
+  int rows_dim;
+  int zero_if_empty;
 };
+
+constexpr int kRowsNone = 0;
+constexpr int kRowsM = 1;
+constexpr int kRowsK = 2;
 
 constexpr int kDepNone = 0;
 constexpr int kDepBeforeLoads = 1;
@@ -140,7 +154,7 @@ struct FwdStatsEpi {
 
   __device__ static void tile(const Params& p, const GemmArgs&, int m_base, int nb,
                               uint32_t taddr, int q, int lane, uint8_t*, const CUtensorMap*,
-                              uint32_t tempty, int&) {
+                              uint32_t tempty, int&, bool) {
     const int row = m_base + q * 32 + lane;
     const bool row_ok = row < p.N;
     const int col0 = nb * BN;
@@ -211,7 +225,7 @@ struct DzEpi {
 
   __device__ static void tile(const Params& p, const GemmArgs&, int m_base, int nb,
                               uint32_t taddr, int q, int lane, uint8_t* stg,
-                              const CUtensorMap* out, uint32_t tempty, int& nstore) {
+                              const CUtensorMap* out, uint32_t tempty, int& nstore, bool) {
     // 64-column chunks whose store box starts inside the block (warp-uniform)
     const int y0 = m_base + q * 32;
     const int rem = p.cols - nb * BN;
@@ -282,6 +296,9 @@ struct DzEpi {
 // Tile * g -> fp32 output rows [out_row0 + m]: TMA store, or TMA reduce-add
 // when `reduce` (accumulation across chunks of the split reduction dimension).
 // g = grad_output * grad_scale, divided by max(n, 1) for 'mean'.
+// With row_map set, output row r is row row_map[r] of out_ptr (row stride ld)
+// and only rows r < *rows_valid exist: the tile is written with vector stores
+// (reduce: read, add, write; each element has one writer per launch).
 struct StoreEpi {
   struct Params {
     int out_row0;
@@ -292,6 +309,10 @@ struct StoreEpi {
     float grad_scale;
     const long long* n_valid;  // device count of non-ignored rows
     int mean;
+    const int* row_map;          // scatter mode: compact row -> output row
+    const long long* rows_valid; // scatter mode: rows that exist
+    float* out_ptr;              // scatter mode: output base
+    int ld;                      // scatter mode: output row stride (floats)
   };
 
   __device__ static float grad_factor(const Params& p) {
@@ -305,17 +326,50 @@ struct StoreEpi {
 
   __device__ static void tile(const Params& p, const GemmArgs&, int m_base, int nb,
                               uint32_t taddr, int q, int lane, uint8_t* stg,
-                              const CUtensorMap* out, uint32_t tempty, int& nstore) {
-    // 32-column chunks whose store box starts inside the output (warp-uniform)
+                              const CUtensorMap* out, uint32_t tempty, int& nstore,
+                              bool empty) {
     const int y = p.out_row0 + m_base + q * 32;
+    int y_end = p.y_limit;
+    if (p.row_map != nullptr) y_end = static_cast<int>(min(static_cast<long long>(y_end), *p.rows_valid));
+    // 32-column chunks whose store box starts inside the output (warp-uniform)
     const int rem = p.x_limit - nb * BN;
-    const int nch = (y >= p.y_limit || rem <= 0) ? 0 : min(BN / 32, (rem + 31) / 32);
+    const int nch = (y >= y_end || rem <= 0) ? 0 : min(BN / 32, (rem + 31) / 32);
     if (nch == 0) {
       release_tmem(tempty, lane);
       return;
     }
+    const float g = empty ? 0.0f : grad_factor(p);  // an empty K range contributes zeros
+    if (p.row_map != nullptr) {
+      const int r = y + lane;
+      const bool live = r < y_end;
+      float* dst = p.out_ptr + static_cast<size_t>(live ? p.row_map[r] : 0) * p.ld + nb * BN;
+#pragma unroll 1
+      for (int c = 0; c < nch; ++c) {
+        uint32_t v[32];
+        tmem_ld_x32(taddr + c * 32, v);
+        tmem_ld_wait();
+        if (c == nch - 1) release_tmem(tempty, lane);
+        if (live) {
+#pragma unroll
+          for (int j4 = 0; j4 < 8; ++j4) {
+            if (nb * BN + c * 32 + 4 * j4 >= p.x_limit) break;  // x_limit is a multiple of 4
+            float4 o = make_float4(__uint_as_float(v[4 * j4]) * g, __uint_as_float(v[4 * j4 + 1]) * g,
+                                   __uint_as_float(v[4 * j4 + 2]) * g, __uint_as_float(v[4 * j4 + 3]) * g);
+            float4* d4 = reinterpret_cast<float4*>(dst + c * 32) + j4;
+            if (p.reduce) {
+              const float4 a = *d4;
+              o.x += a.x;
+              o.y += a.y;
+              o.z += a.z;
+              o.w += a.w;
+            }
+            *d4 = o;
+          }
+        }
+      }
+      return;
+    }
     const uint32_t stg_u32 = smem_u32(stg);
-    const float g = grad_factor(p);
 #pragma unroll 1
     for (int c = 0; c < nch; ++c) {
       uint32_t r[32];
@@ -436,8 +490,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   // The next kernel on the stream may be scheduled as SMs free up; it waits
   // for this one wherever it depends on it.
   griddep_launch_dependents();
-  const int tiles0 = g0.m_tiles * g0.n_tiles;
-  const int num_tiles = tiles0 + g1.m_tiles * g1.n_tiles;
+  // Token-row bounds known only on the device (the same in every thread).
+  auto bound_rows = [](GemmArgs g) {
+    if (g.rows_valid != nullptr && g.rows_dim != kRowsNone) {
+      long long eff = *g.rows_valid - g.rows_base;
+      eff = eff < 0 ? 0 : (eff > g.rows_host ? g.rows_host : eff);
+      if (g.rows_dim == kRowsM) {
+        g.m_tiles = static_cast<int>((eff + Cfg::kUnitRows - 1) / Cfg::kUnitRows);
+      } else {
+        g.k_blocks = static_cast<int>((eff + BK - 1) / BK);
+        if (g.k_blocks == 0 && !g.zero_if_empty) g.m_tiles = 0;
+      }
+    }
+    return g;
+  };
+  const GemmArgs a0 = bound_rows(g0);
+  const GemmArgs a1 = bound_rows(g1);
+  const int tiles0 = a0.m_tiles * a0.n_tiles;
+  const int num_tiles = tiles0 + a1.m_tiles * a1.n_tiles;
   const int unit = blockIdx.x / kCG;  // CTA (kCG = 1) or CTA pair (kCG = 2)
   const int n_units = gridDim.x / kCG;
   volatile int* abort_flag = &abort_sh;
@@ -445,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // problem, its args and the tile's coordinates for global tile index t
   auto locate = [&](int t, int& prob, int& mb, int& nb) {
     prob = (t < tiles0) ? 0 : 1;
-    tile_coords(prob ? t - tiles0 : t, prob ? g1 : g0, mb, nb);
+    tile_coords(prob ? t - tiles0 : t, prob ? a1 : a0, mb, nb);
   };
 
   // ---- tile hand-out.  The leader's producer thread picks each next tile
@@ -506,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok || tile >= num_tiles) break;
         int prob, mb, nb;
         locate(tile, prob, mb, nb);
-        const GemmArgs& g = prob ? g1 : g0;
+        const GemmArgs& g = prob ? a1 : a0;
         const CUtensorMap* mA = prob ? &tmA1 : &tmA0;
         const CUtensorMap* mB = prob ? &tmB1 : &tmB0;
         const bool a_mn = prob ? kAMn1 : kAMn0;
@@ -581,7 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok || tile >= num_tiles) break;
         const int prob = (tile < tiles0) ? 0 : 1;
-        const int k_blocks = prob ? g1.k_blocks : g0.k_blocks;
+        const int k_blocks = prob ? a1.k_blocks : a0.k_blocks;
         const uint32_t idesc = prob ? idesc1 : idesc0;
         const bool a_mn = prob ? kAMn1 : kAMn0;
         const bool b_mn = prob ? kBMn1 : kBMn0;
@@ -674,8 +744,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tempty_local = smem_u32(&bar_tempty[acc]);
       const uint32_t tempty = (kCG == 1) ? tempty_local : mapa_shared(tempty_local, 0);
       const int m_base = mb * Cfg::kUnitRows + static_cast<int>(rank) * BM;
-      Epi::tile(prob ? ep1 : ep0, prob ? g1 : g0, m_base, nb, taddr, q, lane, stg,
-                prob ? &tmOut1 : &tmOut0, tempty, nstore);
+      const GemmArgs& ga = prob ? a1 : a0;
+      Epi::tile(prob ? ep1 : ep0, ga, m_base, nb, taddr, q, lane, stg, prob ? &tmOut1 : &tmOut0,
+                tempty, nstore, ga.k_blocks == 0);
     }
     if (lane == 0) {
       bulk_wait_group_all();

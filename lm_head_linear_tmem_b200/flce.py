@@ -115,17 +115,30 @@ def backward(hidden: torch.Tensor, weight: torch.Tensor, labels: torch.Tensor,
              ignore_index: int = -100, softcap: float = 0.0, reduction: str = "sum",
              workspace: Optional[torch.Tensor] = None,
              d_hidden: Optional[torch.Tensor] = None, d_weight: Optional[torch.Tensor] = None,
+             accumulate_d_hidden: bool = False, accumulate_d_weight: bool = False,
              check_status: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+    """dHidden [N, H] and dWeight [V, H] (float32).  With accumulate_* the
+    gradient is added into the given d_hidden / d_weight instead of
+    overwriting them (e.g. over the micro-batches of one optimizer step)."""
     h2, w, y = _prep(hidden, weight, labels)
     N, H = h2.shape
     V = w.shape[0]
     dev = h2.device
     if workspace is None:
         workspace = alloc_workspace(N, H, V, h2.dtype, dev)
+    for name, t, acc, shape in (("d_hidden", d_hidden, accumulate_d_hidden, (N, H)),
+                                ("d_weight", d_weight, accumulate_d_weight, (V, H))):
+        if acc and t is None:
+            raise ValueError(f"accumulating needs an existing {name}")
+        if t is not None and (tuple(t.shape) != shape or t.dtype != torch.float32
+                              or not t.is_contiguous() or t.device != dev):
+            raise ValueError(f"{name} must be a contiguous float32 {list(shape)} tensor on {dev}")
     if d_hidden is None:
         d_hidden = torch.empty((N, H), dtype=torch.float32, device=dev)
     if d_weight is None:
         d_weight = torch.empty((V, H), dtype=torch.float32, device=dev)
+    flags = ((_native.ACCUMULATE_DHIDDEN if accumulate_d_hidden else 0)
+             | (_native.ACCUMULATE_DWEIGHT if accumulate_d_weight else 0))
     if grad_output is not None:
         grad_output = grad_output.reshape(()).to(device=dev, dtype=torch.float32).contiguous()
     if num_valid is not None:
@@ -134,7 +147,7 @@ def backward(hidden: torch.Tensor, weight: torch.Tensor, labels: torch.Tensor,
     st = _lib().flce_backward(_ptr(h2), _ptr(w), _ptr(y), _ptr(lse), N, H, V, int(ignore_index),
                               float(softcap), _REDUCTIONS[reduction], _DTYPES[h2.dtype],
                               _ptr(grad_output), float(grad_scale), _ptr(num_valid),
-                              _ptr(d_hidden), _ptr(d_weight), _ptr(workspace),
+                              _ptr(d_hidden), _ptr(d_weight), flags, _ptr(workspace),
                               workspace.numel(), _stream(dev))
     _native.check(st, "flce_backward")
     if check_status:

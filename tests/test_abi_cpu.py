@@ -55,8 +55,9 @@ def test_workspace_bytes(lib):
     assert tiny > 0 and tiny % 256 == 0
     big = ws(16384, 4096, 131072, 0)
     # forward partials: 512 vocab tiles x 16384 rows x (m, s) fp32 = 64 MiB;
-    # backward dZ block: 4096 x 8192 bf16 = 64 MiB
-    assert 64 * 2 ** 20 <= big < 66 * 2 ** 20
+    # backward: compact hidden 16384 x 4096 bf16 = 128 MiB + dZ block
+    # 4096 x 8192 bf16 = 64 MiB + row-compaction arrays
+    assert 192 * 2 ** 20 <= big < 194 * 2 ** 20
     assert ws(0, 64, 512, 0) > 0
     assert ws(64, 64, 512, 1) > 0
 
@@ -85,10 +86,13 @@ def test_argument_errors_are_synchronous(lib):
     assert _fwd(lib, labels=FAKE + 4) == ARG
     assert _fwd(lib, ws_size=1024) == WS
     assert _fwd(lib, loss=None) == ARG
+    wsb = lib.flce_workspace_bytes(64, 64, 512, 0)
     bad_bwd = lib.flce_backward(FAKE, FAKE, FAKE, FAKE, 64, 64, 512, -100, 0.0, 0, 0, None,
-                                float("nan"), None, FAKE, FAKE, FAKE,
-                                lib.flce_workspace_bytes(64, 64, 512, 0), None)
+                                float("nan"), None, FAKE, FAKE, 0, FAKE, wsb, None)
     assert bad_bwd == ARG
+    bad_flags = lib.flce_backward(FAKE, FAKE, FAKE, FAKE, 64, 64, 512, -100, 0.0, 0, 0, None,
+                                  1.0, None, FAKE, FAKE, 4, FAKE, wsb, None)
+    assert bad_flags == ARG
     assert lib.flce_get_status(None, None) == ARG
 
 

@@ -113,39 +113,44 @@ def test_fullsize_sampled(name):
 
 def test_microbatch_token_weighted_scale():
     """4 micro-batches of 4096 tokens, micro-batch 1 all ignored; 'sum' with
-    grad_scale = 1 / sum_k n_k; dWeight accumulated over the micro-batches."""
+    grad_scale = 1 / sum_k n_k; dWeight accumulated over the micro-batches by
+    the library (accumulate flag), as a trainer does within one step."""
     gold = golden("microbatch")
     inp = fi.make_inputs("microbatch")
     w = inp.workload
     h, W, y = device_inputs(inp)
     n_tot = int(gold["num_valid"])
     gs = 1.0 / n_tot
-    dw_acc = torch.zeros(w.V, w.H, dtype=torch.float32, device="cuda")
+    dw_acc = torch.empty(w.V, w.H, dtype=torch.float32, device="cuda")
     dh_all = torch.empty(w.N, w.H, dtype=torch.float32, device="cuda")
     lse_all = torch.empty(w.N, dtype=torch.float32, device="cuda")
     total = 0.0
     ntok = 0
     ws = flce.alloc_workspace(w.N // w.microbatches, w.H, w.V, torch.bfloat16, "cuda")
-    for k, sl in enumerate(inp.microbatch_slices()):
-        f = flce.forward(h[sl], W, y[sl], IGN, 0.0, "sum", workspace=ws, check_status=True)
-        dh, dw = flce.backward(h[sl], W, y[sl], f.lse, grad_scale=gs, workspace=ws,
-                               check_status=True)
+    slices = inp.microbatch_slices()
+    for k, sl in enumerate(slices):
+        f = flce.forward(h[sl], W, y[sl], IGN, 0.0, "sum", workspace=ws, lse=lse_all[sl],
+                         check_status=True)
+        flce.backward(h[sl], W, y[sl], f.lse, grad_scale=gs, workspace=ws, d_hidden=dh_all[sl],
+                      d_weight=dw_acc, accumulate_d_weight=(k > 0), check_status=True)
         lk = f.loss.item()
         nk = int(f.num_tokens.item())
         assert nk == int(gold["mb_count"][k])
         G.check_loss(lk, float(gold["mb_loss"][k]))
         if k == w.empty_microbatch:
             assert lk == 0.0 and nk == 0
-            assert bool(torch.all(dh == 0)) and bool(torch.all(dw == 0))
-        assert bool(torch.isfinite(dw).all())
+            assert bool(torch.all(dh_all[sl] == 0))
         total += lk
         ntok += nk
-        dw_acc += dw
-        dh_all[sl] = dh
-        lse_all[sl] = f.lse
-        del dw
     assert ntok == n_tot
     G.check_loss(total, float(gold["loss"]))
+    # the all-ignored micro-batch on its own adds exactly nothing to dWeight
+    sl = slices[w.empty_microbatch]
+    _, dw_empty = flce.backward(h[sl], W, y[sl], lse_all[sl], grad_scale=gs, workspace=ws,
+                                check_status=True)
+    assert bool(torch.all(dw_empty == 0))
+    del dw_empty
+    assert bool(torch.isfinite(dw_acc).all())
     torch.cuda.synchronize()
     _check_sampled(inp, gold, lse_all.cpu().numpy(), dh_all.cpu().numpy(),
                    dw_acc.cpu().numpy(), gs, seed=5)

@@ -157,3 +157,45 @@ def test_repeated_calls_are_deterministic():
     assert a["loss"] == b["loss"]
     assert np.array_equal(a["lse"], b["lse"])
     assert np.array_equal(a["dh"], b["dh"]) and np.array_equal(a["dw"], b["dw"])
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_accumulate_flags(dtype):
+    inp = G.small_inputs(N=4200, H=136, V=9000, seed=15, n_ign=300, w_std=0.1)
+    if dtype == "bf16":
+        h, W = G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits)
+    else:
+        inp = G.small_inputs(N=96, H=64, V=700, seed=15, n_ign=10, w_std=0.1)
+        h, W = G.f32_tensor(inp.hidden_raw), G.f32_tensor(inp.weight_raw)
+    y = G.labels_tensor(inp.labels)
+    f = flce.forward(h, W, y, check_status=True)
+    dh1, dw1 = flce.backward(h, W, y, f.lse, grad_scale=0.5, check_status=True)
+    dh2, dw2 = dh1.clone(), dw1.clone()
+    flce.backward(h, W, y, f.lse, grad_scale=0.5, d_hidden=dh2, d_weight=dw2,
+                  accumulate_d_hidden=True, accumulate_d_weight=True, check_status=True)
+    torch.cuda.synchronize()
+    assert G.rel_l2(dh2.cpu().numpy(), 2 * dh1.cpu().numpy().astype(np.float64)) <= 1e-6
+    assert G.rel_l2(dw2.cpu().numpy(), 2 * dw1.cpu().numpy().astype(np.float64)) <= 1e-6
+    # accumulate only dWeight: dHidden is overwritten
+    dh3, dw3 = dh1.clone(), dw1.clone()
+    flce.backward(h, W, y, f.lse, grad_scale=0.5, d_hidden=dh3, d_weight=dw3,
+                  accumulate_d_weight=True, check_status=True)
+    assert torch.equal(dh3, dh1)
+
+
+def test_microbatch_accumulation_matches_full_batch():
+    inp = G.small_inputs(N=4400, H=128, V=9000, seed=16, n_ign=400, w_std=0.1)
+    h, W, y = (G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
+               G.labels_tensor(inp.labels))
+    n = int((inp.labels != IGN).sum())
+    f = flce.forward(h, W, y)
+    dh_full, dw_full = flce.backward(h, W, y, f.lse, grad_scale=1.0 / n)
+    dw_acc = torch.empty_like(dw_full)
+    dh_acc = torch.empty_like(dh_full)
+    for k, sl in enumerate([slice(0, 1500), slice(1500, 4400)]):
+        fk = flce.forward(h[sl], W, y[sl], check_status=True)
+        flce.backward(h[sl], W, y[sl], fk.lse, grad_scale=1.0 / n, d_hidden=dh_acc[sl],
+                      d_weight=dw_acc, accumulate_d_weight=(k > 0), check_status=True)
+    torch.cuda.synchronize()
+    assert G.rel_l2(dw_acc.cpu().numpy(), dw_full.cpu().numpy().astype(np.float64)) <= 1e-5
+    assert G.rel_l2(dh_acc.cpu().numpy(), dh_full.cpu().numpy().astype(np.float64)) <= 1e-6
