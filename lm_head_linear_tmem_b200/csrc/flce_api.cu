@@ -193,10 +193,13 @@ int64_t bwd_launches(int64_t N, int64_t V) {
 }
 
 // Backward workspace: header | tile counters | row compaction (permutation,
-// compact labels and lse, per-block counts, valid count) | compact hidden
-// [N, H] bf16 | dZ block.
+// compact labels and lse, per-block counts, valid count) | label sort (two
+// key/value buffers, digit counts) | label residuals | compact hidden [N, H]
+// bf16 | dZ block, whose space the dWeight label correction's run pieces
+// reuse once the GEMMs are done.
 struct BwdLayout {
-  size_t counters, perm, labels_c, lse_c, block_valid, n_valid_c, hidden_c, gblock, end;
+  size_t counters, perm, labels_c, lse_c, block_valid, n_valid_c, keys0, keys1, vals0, vals1,
+      hist, resid, hidden_c, gblock, part, end;
 };
 
 BwdLayout bwd_layout(int64_t N, int64_t H, int64_t V) {
@@ -215,11 +218,20 @@ BwdLayout bwd_layout(int64_t N, int64_t H, int64_t V) {
   L.block_valid = off;
   off = align_up(off + 4 * nblk, 256);
   L.n_valid_c = off;
-  off = align_up(off + 8, 1024);
+  off = align_up(off + 8, 256);
+  for (size_t* b : {&L.keys0, &L.keys1, &L.vals0, &L.vals1, &L.resid}) {
+    *b = off;
+    off = align_up(off + 4 * static_cast<size_t>(N), 256);
+  }
+  L.hist = off;
+  off = align_up(off + 4 * static_cast<size_t>(kRadixBuckets) * nblk, 1024);
   L.hidden_c = off;
   off = align_up(off + 2 * static_cast<size_t>(N) * static_cast<size_t>(H), 1024);
   L.gblock = off;
-  off += static_cast<size_t>(c.tc) * c.vc * 2 + 1024;
+  L.part = off;
+  const size_t nseg = static_cast<size_t>((N + kFixSeg - 1) / kFixSeg);
+  off += std::max(static_cast<size_t>(c.tc) * c.vc * 2 + 1024,
+                  nseg * 2 * static_cast<size_t>(H) * 4);
   L.end = off;
   return L;
 }
@@ -522,6 +534,7 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
   const float* lsev = lse;
   int* perm = nullptr;
   const long long* rows_valid = nullptr;
+  float* resid = nullptr;  // label-entry residuals (compact mode: label-sorted rows)
   if (compact) {
     perm = reinterpret_cast<int*>(w + BL.perm);
     int64_t* labels_c = reinterpret_cast<int64_t*>(w + BL.labels_c);
@@ -536,12 +549,44 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
     });
     if (e == cudaSuccess)
       e = launch(kHelper, st, [&] {
-        compact_scan_kernel<<<1, kCompactThreads, 0, st>>>(block_valid, nblk, n_valid_c);
+        exclusive_scan_kernel<<<1, kCompactThreads, 0, st>>>(block_valid, nblk, n_valid_c);
       });
+    uint32_t* keys[2] = {reinterpret_cast<uint32_t*>(w + BL.keys0),
+                         reinterpret_cast<uint32_t*>(w + BL.keys1)};
+    int* vals[2] = {reinterpret_cast<int*>(w + BL.vals0), reinterpret_cast<int*>(w + BL.vals1)};
     if (e == cudaSuccess)
       e = launch(kHelper, st, [&] {
         compact_scatter_kernel<<<nblk, kCompactThreads, 0, st>>>(
-            labels, lse, n, ignore_index, block_valid, n_valid_c, perm, labels_c, lse_c);
+            labels, lse, n, ignore_index, block_valid, n_valid_c, perm, labels_c, lse_c, V,
+            keys[0], vals[0]);
+      });
+    // Valid rows in (label, token) order: keys are labels, or V for a label
+    // outside [0, V), so ceil(bits(V) / 8) passes of 8 bits sort them.
+    int key_bits = 0;
+    while ((V >> key_bits) != 0) ++key_bits;
+    const int passes = (key_bits + 7) / 8;
+    int* hist = reinterpret_cast<int*>(w + BL.hist);
+    for (int ps = 0; ps < passes && e == cudaSuccess; ++ps) {
+      const int src = ps & 1, shift = 8 * ps;
+      e = launch(kHelper, st, [&] {
+        radix_hist_kernel<<<nblk, kCompactThreads, 0, st>>>(keys[src], n_valid_c, shift, nblk,
+                                                              hist);
+      });
+      if (e == cudaSuccess)
+        e = launch(kHelper, st, [&] {
+          exclusive_scan_kernel<<<1, kCompactThreads, 0, st>>>(hist, kRadixBuckets * nblk,
+                                                               nullptr);
+        });
+      if (e == cudaSuccess)
+        e = launch(kHelper, st, [&] {
+          radix_scatter_kernel<<<nblk, kCompactThreads, 0, st>>>(
+              keys[src], vals[src], keys[src ^ 1], vals[src ^ 1], n_valid_c, shift, nblk, hist);
+        });
+    }
+    if (e == cudaSuccess)
+      e = launch(kHelper, st, [&] {
+        apply_label_order_kernel<<<nblk, kCompactThreads, 0, st>>>(
+            keys[passes & 1], vals[passes & 1], lse, n_valid_c, perm, labels_c, lse_c);
       });
     if (e == cudaSuccess)
       e = launch(kHelper, st, [&] {
@@ -554,6 +599,7 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
     hid = hidden_c;
     lab = labels_c;
     lsev = lse_c;
+    resid = reinterpret_cast<float*>(w + BL.resid);
     rows_valid = n_valid_c;
     if (n_valid_is_count) n_valid = n_valid_c;  // the library's own count serves both
   }
@@ -606,12 +652,13 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
       cudaError_t e;
       const GemmProblem pz{&t_hid_k, &t_w_k, &t_g_store, rows, gz};
       if (softcap > 0.f) {
-        DzEpi<true>::Params ep{lab, lsev, ignore_index, static_cast<int>(t0), rows,
-                               static_cast<int>(v0), cols, softcap, 1.0f / softcap};
+        DzEpi<true>::Params ep{lab,  lsev,    ignore_index, static_cast<int>(t0),
+                               rows, static_cast<int>(v0), cols, softcap, 1.0f / softcap,
+                               resid};
         e = run_gemm<DzEpi<true>, false, false>(d, kSlotDzCap, kBwdDz, pz, ep, nullptr, ep, st);
       } else {
-        DzEpi<false>::Params ep{lab, lsev, ignore_index, static_cast<int>(t0), rows,
-                                static_cast<int>(v0), cols, 0.f, 0.f};
+        DzEpi<false>::Params ep{lab,  lsev, ignore_index, static_cast<int>(t0), rows,
+                                static_cast<int>(v0), cols, 0.f, 0.f, resid};
         e = run_gemm<DzEpi<false>, false, false>(d, kSlotDz, kBwdDz, pz, ep, nullptr, ep, st);
       }
       if (e != cudaSuccess) return cuda_fail(e);
@@ -631,9 +678,13 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
       gh.rows_host = rows;
       gh.rows_dim = kRowsM;
       gh.dep_wait = kDepBeforeLoads;  // reads the dZ block written just before
+      // the last vocab chunk's dHidden epilogue also adds the exact label term
+      const bool last_v = v0 + ck.vc >= V;
       StoreEpi::Params eh{static_cast<int>(t0), (v0 > 0 || acc_dh) ? 1 : 0, static_cast<int>(H),
                           static_cast<int>(N), grad_output, grad_scale, n_valid, mean,
-                          perm, rows_valid, d_hidden, static_cast<int>(H)};
+                          perm, rows_valid, d_hidden, static_cast<int>(H),
+                          last_v ? resid : nullptr, lab,
+                          static_cast<const __nv_bfloat16*>(weight), static_cast<long long>(V)};
 
       // 3) dWeight[v0:v0+cols] (+)= dZ^T . hidden[t0:t0+rows]
       GemmArgs gw{};
@@ -653,7 +704,7 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
       gw.dep_wait = kDepBeforeLoads;
       StoreEpi::Params ew{static_cast<int>(v0), (t0 > 0 || acc_dw) ? 1 : 0, static_cast<int>(H),
                           static_cast<int>(V), grad_output, grad_scale, n_valid, mean,
-                          nullptr, nullptr, nullptr, 0};
+                          nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0};
 
       const GemmProblem ph{&t_g_k, &t_w_mn, &t_dh, rows, gh};
       const GemmProblem pw{&t_g_mn, &t_hid_mn, &t_dw, cols, gw};
@@ -667,6 +718,26 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
       }
       if (e != cudaSuccess) return cuda_fail(e);
     }
+  }
+
+  if (compact) {
+    // dWeight's exact label term, per label run (dHidden's was added above).
+    float* part = reinterpret_cast<float*>(w + BL.part);
+    const dim3 grid(static_cast<unsigned>((N + kFixSeg - 1) / kFixSeg),
+                    static_cast<unsigned>((H + kFixCols - 1) / kFixCols));
+    const int64_t* labels_c = lab;
+    cudaError_t e = launch(kHelper, st, [&] {
+      dw_fix_segments_kernel<<<grid, kFixThreads, 0, st>>>(
+          labels_c, resid, rows_valid, static_cast<const __nv_bfloat16*>(hid),
+          static_cast<int>(H), V, d_weight, part, grad_output, grad_scale, n_valid, mean);
+    });
+    if (e == cudaSuccess)
+      e = launch(kHelper, st, [&] {
+        dw_fix_runs_kernel<<<grid, kFixThreads, 0, st>>>(labels_c, rows_valid,
+                                                         static_cast<int>(H), V, d_weight, part,
+                                                         grad_output, grad_scale, n_valid, mean);
+      });
+    if (e != cudaSuccess) return cuda_fail(e);
   }
   return FLCE_OK;
 }

@@ -172,18 +172,18 @@ __global__ void __launch_bounds__(kCompactThreads)
   }
 }
 
-// One block: exclusive prefix sum of the per-block counts (in place) and the
-// total number of valid rows.
+// One block: exclusive prefix sum of a[0..n) in place (the per-block valid
+// counts, or a radix pass's digit counts), and the total when `total` is set.
 __global__ void __launch_bounds__(kCompactThreads)
-    compact_scan_kernel(int* __restrict__ block_valid, int nblk, long long* __restrict__ n_valid) {
+    exclusive_scan_kernel(int* __restrict__ a, int n, long long* __restrict__ total) {
   __shared__ int carry;
   __shared__ int warp_sum[kCompactThreads / 32];
   if (threadIdx.x == 0) carry = 0;
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int base = 0; base < nblk; base += kCompactThreads) {
+  for (int base = 0; base < n; base += kCompactThreads) {
     const int b = base + threadIdx.x;
-    const int x = (b < nblk) ? block_valid[b] : 0;
+    const int x = (b < n) ? a[b] : 0;
     int incl = x;  // inclusive scan within the warp
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, incl, o);
@@ -195,11 +195,11 @@ __global__ void __launch_bounds__(kCompactThreads)
     for (int w = 0; w < warp; ++w) before += warp_sum[w];
     const int excl = carry + before + incl - x;
     __syncthreads();
-    if (b < nblk) block_valid[b] = excl;
+    if (b < n) a[b] = excl;
     if (threadIdx.x == kCompactThreads - 1) carry = excl + x;
     __syncthreads();
   }
-  if (threadIdx.x == 0) *n_valid = carry;
+  if (threadIdx.x == 0 && total != nullptr) *total = carry;
 }
 
 // perm[j], and the compact labels and lse of every compact row: valid rows keep
@@ -208,7 +208,9 @@ __global__ void __launch_bounds__(kCompactThreads)
     compact_scatter_kernel(const int64_t* __restrict__ labels, const float* __restrict__ lse,
                            int N, int64_t ignore_index, const int* __restrict__ block_offset,
                            const long long* __restrict__ n_valid, int* __restrict__ perm,
-                           int64_t* __restrict__ labels_c, float* __restrict__ lse_c) {
+                           int64_t* __restrict__ labels_c, float* __restrict__ lse_c,
+                           int64_t V, uint32_t* __restrict__ sort_keys,
+                           int* __restrict__ sort_vals) {
   __shared__ int warp_sum[kCompactThreads / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int i = blockIdx.x * kCompactThreads + threadIdx.x;
@@ -225,7 +227,217 @@ __global__ void __launch_bounds__(kCompactThreads)
     perm[j] = i;
     labels_c[j] = v ? y : ignore_index;
     lse_c[j] = v ? lse[i] : 0.f;
+    if (v) {  // labels outside [0, V) share the key V and are sorted last
+      sort_keys[j] = static_cast<uint32_t>((y >= 0 && y < V) ? y : V);
+      sort_vals[j] = i;
+    }
   }
+}
+
+// ------------------------------------------------------------------ label sort
+// The valid rows are then put in (label, row) order by a stable LSD radix sort
+// on 8-bit digits of the label, so the rows of each label are contiguous and
+// the per-label sums below have a fixed order.  Only the first *n_valid
+// entries take part.
+constexpr int kRadixBuckets = 256;
+
+// Per-block digit counts, digit-major: hist[digit * nblk + block].
+__global__ void __launch_bounds__(kCompactThreads)
+    radix_hist_kernel(const uint32_t* __restrict__ keys, const long long* __restrict__ n_valid,
+                      int shift, int nblk, int* __restrict__ hist) {
+  __shared__ int h[kRadixBuckets];
+  for (int t = threadIdx.x; t < kRadixBuckets; t += blockDim.x) h[t] = 0;
+  __syncthreads();
+  const long long j = static_cast<long long>(blockIdx.x) * kCompactThreads + threadIdx.x;
+  if (j < *n_valid) atomicAdd(&h[(keys[j] >> shift) & (kRadixBuckets - 1)], 1);
+  __syncthreads();
+  for (int t = threadIdx.x; t < kRadixBuckets; t += blockDim.x) hist[t * nblk + blockIdx.x] = h[t];
+}
+
+// Stable scatter of one radix pass: an element's place is its digit's block
+// offset plus the number of equal digits before it in the block (earlier
+// warps, then earlier lanes of its warp).
+__global__ void __launch_bounds__(kCompactThreads)
+    radix_scatter_kernel(const uint32_t* __restrict__ keys_in, const int* __restrict__ vals_in,
+                         uint32_t* __restrict__ keys_out, int* __restrict__ vals_out,
+                         const long long* __restrict__ n_valid, int shift, int nblk,
+                         const int* __restrict__ offsets) {
+  __shared__ int wcnt[kCompactThreads / 32][kRadixBuckets];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int t = threadIdx.x; t < (kCompactThreads / 32) * kRadixBuckets; t += blockDim.x)
+    (&wcnt[0][0])[t] = 0;
+  __syncthreads();
+  const long long j = static_cast<long long>(blockIdx.x) * kCompactThreads + threadIdx.x;
+  const bool live = j < *n_valid;
+  const uint32_t key = live ? keys_in[j] : 0u;
+  const int dg = live ? static_cast<int>((key >> shift) & (kRadixBuckets - 1)) : kRadixBuckets;
+  const unsigned peers = __match_any_sync(0xffffffffu, dg);
+  const int rank_w = __popc(peers & ((1u << lane) - 1u));
+  if (live && rank_w == 0) wcnt[warp][dg] = __popc(peers);
+  __syncthreads();
+  if (threadIdx.x < kRadixBuckets) {
+    int run = 0;
+    for (int w = 0; w < kCompactThreads / 32; ++w) {
+      const int c = wcnt[w][threadIdx.x];
+      wcnt[w][threadIdx.x] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  if (live) {
+    const int dst = offsets[dg * nblk + blockIdx.x] + wcnt[warp][dg] + rank_w;
+    keys_out[dst] = key;
+    vals_out[dst] = vals_in[j];
+  }
+}
+
+// The sorted valid rows become compact rows 0..n_valid-1.
+__global__ void __launch_bounds__(kCompactThreads)
+    apply_label_order_kernel(const uint32_t* __restrict__ keys, const int* __restrict__ vals,
+                             const float* __restrict__ lse, const long long* __restrict__ n_valid,
+                             int* __restrict__ perm, int64_t* __restrict__ labels_c,
+                             float* __restrict__ lse_c) {
+  const long long j = static_cast<long long>(blockIdx.x) * kCompactThreads + threadIdx.x;
+  if (j >= *n_valid) return;
+  const int i = vals[j];
+  perm[j] = i;
+  labels_c[j] = static_cast<int64_t>(keys[j]);
+  lse_c[j] = lse[i];
+}
+
+// ------------------------------------------------------------------ label-entry residuals
+// The dZ block holds bf16(dZ/g).  For the label entry of each valid row, which
+// dominates the row's gradient, the rounding residual e = d - bf16(d) (exact in
+// fp32) is recorded by the dZ epilogue and added back here in fp32:
+//   dHidden[row]   += g * e * W[label]
+//   dWeight[label] += g * sum over the label's rows (in order) of e * hidden[row]
+__device__ __forceinline__ float backward_grad_factor(const float* grad_output, float grad_scale,
+                                                      const long long* n_valid_for_mean,
+                                                      int mean) {
+  float g = (grad_output != nullptr ? grad_output[0] : 1.0f) * grad_scale;
+  if (mean) {
+    const long long n = *n_valid_for_mean;
+    g = g / static_cast<float>(n > 0 ? n : 1);
+  }
+  return g;
+}
+
+// dWeight part, deterministic: the valid compact rows are in label order, so
+// each label's rows form one run.  Phase 1 cuts the rows into segments of
+// kFixSeg and sums e * hidden over each run piece in row order; a run that
+// lies inside one segment is added to dWeight at once, a run crossing a
+// segment boundary leaves its piece in part[seg][slot] (slot 0: the segment's
+// first run, begun in an earlier segment; slot 1: its last run, going on into
+// the next).  Phase 2 lets the segment where such a run begins add its pieces
+// in segment order.  Blocks cover kFixCols columns, two per thread.
+constexpr int kFixSeg = 64;
+constexpr int kFixCols = 256;
+constexpr int kFixThreads = kFixCols / 2;
+
+__device__ __forceinline__ void dw_fix_add(float* d_weight, int64_t v, int64_t V, int H, int col,
+                                           float g, float a0, float a1) {
+  if (v < 0 || v >= V) return;  // a label the forward reported as out of range
+  float2* o = reinterpret_cast<float2*>(d_weight + static_cast<size_t>(v) * H + col);
+  float2 cur = *o;
+  cur.x = fmaf(g, a0, cur.x);
+  cur.y = fmaf(g, a1, cur.y);
+  *o = cur;
+}
+
+__global__ void __launch_bounds__(kFixThreads)
+    dw_fix_segments_kernel(const int64_t* __restrict__ labels_c, const float* __restrict__ resid,
+                           const long long* __restrict__ rows_valid,
+                           const __nv_bfloat16* __restrict__ hidden_c, int H, int64_t V,
+                           float* __restrict__ d_weight, float* __restrict__ part,
+                           const float* grad_output, float grad_scale,
+                           const long long* n_valid_for_mean, int mean) {
+  const long long nv = *rows_valid;
+  const long long s0 = static_cast<long long>(blockIdx.x) * kFixSeg;
+  if (s0 >= nv) return;
+  const int n = static_cast<int>(min(static_cast<long long>(kFixSeg), nv - s0));
+  __shared__ int64_t lab[kFixSeg];
+  __shared__ float es[kFixSeg];
+  __shared__ int64_t lab_before, lab_after;
+  for (int t = threadIdx.x; t < n; t += blockDim.x) {
+    lab[t] = labels_c[s0 + t];
+    es[t] = resid[s0 + t];
+  }
+  if (threadIdx.x == 0) {
+    lab_before = s0 > 0 ? labels_c[s0 - 1] : INT64_MIN;
+    lab_after = s0 + n < nv ? labels_c[s0 + n] : INT64_MIN;
+  }
+  __syncthreads();
+  const int col = blockIdx.y * kFixCols + 2 * threadIdx.x;
+  if (col >= H) return;  // H is even
+  const float g = backward_grad_factor(grad_output, grad_scale, n_valid_for_mean, mean);
+  float* part_seg = part + static_cast<size_t>(blockIdx.x) * 2 * H;
+  const __nv_bfloat16* hrow = hidden_c + static_cast<size_t>(s0) * H + col;
+  int64_t cur = lab[0];
+  bool begun_before = (cur == lab_before);
+  float a0 = 0.f, a1 = 0.f;
+  for (int kb = 0; kb < n; kb += 8) {
+    float2 hv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (kb + i < n)
+        hv[i] = __bfloat1622float2(
+            *reinterpret_cast<const __nv_bfloat162*>(hrow + static_cast<size_t>(kb + i) * H));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (kb + i >= n) break;
+      const int64_t l = lab[kb + i];
+      if (l != cur) {  // the run `cur` ends inside the segment
+        if (begun_before) {
+          part_seg[col] = a0;
+          part_seg[col + 1] = a1;
+        } else {
+          dw_fix_add(d_weight, cur, V, H, col, g, a0, a1);
+        }
+        cur = l;
+        begun_before = false;
+        a0 = a1 = 0.f;
+      }
+      a0 = fmaf(es[kb + i], hv[i].x, a0);
+      a1 = fmaf(es[kb + i], hv[i].y, a1);
+    }
+  }
+  const bool goes_on = (cur == lab_after);
+  if (begun_before) {
+    part_seg[col] = a0;
+    part_seg[col + 1] = a1;
+  } else if (goes_on) {
+    part_seg[H + col] = a0;
+    part_seg[H + col + 1] = a1;
+  } else {
+    dw_fix_add(d_weight, cur, V, H, col, g, a0, a1);
+  }
+}
+
+__global__ void __launch_bounds__(kFixThreads)
+    dw_fix_runs_kernel(const int64_t* __restrict__ labels_c, const long long* __restrict__ rows_valid,
+                       int H, int64_t V, float* __restrict__ d_weight,
+                       const float* __restrict__ part, const float* grad_output, float grad_scale,
+                       const long long* n_valid_for_mean, int mean) {
+  const long long nv = *rows_valid;
+  const long long s0 = static_cast<long long>(blockIdx.x) * kFixSeg;
+  if (s0 >= nv) return;
+  long long last = min(s0 + kFixSeg, nv) - 1;
+  const int64_t L = labels_c[last];
+  if (last + 1 >= nv || labels_c[last + 1] != L) return;  // the last run ends here
+  if (s0 > 0 && labels_c[s0 - 1] == L) return;           // it began in an earlier segment
+  const int col = blockIdx.y * kFixCols + 2 * threadIdx.x;
+  if (col >= H) return;
+  const float* p = part + static_cast<size_t>(blockIdx.x) * 2 * H;
+  float a0 = p[H + col], a1 = p[H + col + 1];
+  for (long long s = blockIdx.x + 1;; ++s) {
+    p = part + static_cast<size_t>(s) * 2 * H;
+    a0 += p[col];
+    a1 += p[col + 1];
+    last = min((s + 1) * kFixSeg, nv) - 1;
+    if (last + 1 >= nv || labels_c[last + 1] != L) break;
+  }
+  const float g = backward_grad_factor(grad_output, grad_scale, n_valid_for_mean, mean);
+  dw_fix_add(d_weight, L, V, H, col, g, a0, a1);
 }
 
 // Compact hidden: row j < n_valid is hidden[perm[j]]; rows past n_valid are

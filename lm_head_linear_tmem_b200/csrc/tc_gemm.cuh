@@ -209,6 +209,9 @@ struct FwdStatsEpi {
 // in fp32, by the dHidden / dWeight epilogues: folding an arbitrary g into
 // the bf16 value would move the dominant label entry (p - 1 ~ -1, which
 // rounds to -1 almost exactly) off the bf16 grid.
+// With `resid` set, the label entry's rounding residual d - bf16(d) (exact in
+// fp32) is recorded per row, for the fp32 corrections that make the label
+// term of dHidden and dWeight exact.
 template <bool kSoftcap>
 struct DzEpi {
   struct Params {
@@ -221,6 +224,7 @@ struct DzEpi {
     int cols;   // valid vocab columns in this block
     float softcap;
     float inv_softcap;
+    float* resid;  // [token rows] or null
   };
 
   __device__ static void tile(const Params& p, const GemmArgs&, int m_base, int nb,
@@ -269,6 +273,8 @@ struct DzEpi {
             const float u = L * p.inv_softcap;
             d *= fmaf(-u, u, 1.0f);
           }
+          if (p.resid != nullptr && c2 * 64 + jj == y_local)
+            p.resid[p.t0 + row_l] = d - __bfloat162float(__float2bfloat16_rn(d));
           gv[h] = valid ? d : 0.0f;
         }
         __nv_bfloat162 b2 = __floats2bfloat162_rn(gv[0], gv[1]);
@@ -313,6 +319,12 @@ struct StoreEpi {
     const long long* rows_valid; // scatter mode: rows that exist
     float* out_ptr;              // scatter mode: output base
     int ld;                      // scatter mode: output row stride (floats)
+    // scatter mode, dHidden: adds g * resid[r] * W[labels[r]] to row r (the
+    // exact label term; see DzEpi).  Null for no correction.
+    const float* fix_resid;
+    const int64_t* fix_labels;
+    const __nv_bfloat16* fix_w;  // [V, x_limit] row-major
+    long long fix_v;
   };
 
   __device__ static float grad_factor(const Params& p) {
@@ -343,6 +355,15 @@ struct StoreEpi {
       const int r = y + lane;
       const bool live = r < y_end;
       float* dst = p.out_ptr + static_cast<size_t>(live ? p.row_map[r] : 0) * p.ld + nb * BN;
+      float cfix = 0.f;
+      const __nv_bfloat16* wrow = nullptr;
+      if (p.fix_resid != nullptr && live) {
+        const int64_t yl = p.fix_labels[r];
+        if (yl >= 0 && yl < p.fix_v) {
+          cfix = grad_factor(p) * p.fix_resid[r];
+          wrow = p.fix_w + static_cast<size_t>(yl) * p.x_limit + nb * BN;
+        }
+      }
 #pragma unroll 1
       for (int c = 0; c < nch; ++c) {
         uint32_t v[32];
@@ -356,6 +377,15 @@ struct StoreEpi {
             float4 o = make_float4(__uint_as_float(v[4 * j4]) * g, __uint_as_float(v[4 * j4 + 1]) * g,
                                    __uint_as_float(v[4 * j4 + 2]) * g, __uint_as_float(v[4 * j4 + 3]) * g);
             float4* d4 = reinterpret_cast<float4*>(dst + c * 32) + j4;
+            if (wrow != nullptr) {
+              const uint2 wv = *reinterpret_cast<const uint2*>(wrow + c * 32 + 4 * j4);
+              const float2 w01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv.x));
+              const float2 w23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv.y));
+              o.x = fmaf(cfix, w01.x, o.x);
+              o.y = fmaf(cfix, w01.y, o.y);
+              o.z = fmaf(cfix, w23.x, o.z);
+              o.w = fmaf(cfix, w23.y, o.w);
+            }
             if (p.reduce) {
               const float4 a = *d4;
               o.x += a.x;
@@ -712,8 +742,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ---------------- epilogue warps
-    if (g0.dep_wait == kDepBeforeStores) griddep_wait();
+    // ---------------- epilogue warps (they may read what the previous kernel
+    // wrote, so they wait for it in either mode)
+    if (g0.dep_wait != kDepNone) griddep_wait();
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     uint8_t* stg = smem + kStages * Cfg::kStageBytes + (warp - 2) * kStagingPerWarp;
     int it = 0;
