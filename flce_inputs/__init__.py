@@ -91,14 +91,14 @@ WORKLOADS: Dict[str, Workload] = {
         softcap=0.0, reduction="sum", seed=5, microbatches=4, empty_microbatch=1,
         description="N=16384 as 4 micro-batches of 4096, micro-batch 1 all ignored, "
                     "others 30% ignored, sum with token-weighted grad scale"),
-    # A smaller problem whose kernel launches have exactly the per-launch
-    # shapes of v131k_zipf (H=4096; 4096-token x 8192-vocab backward chunks),
+    # A smaller problem whose backward launches have exactly the per-launch
+    # shapes of v131k_zipf (H=4096; 8192-token x 16384-vocab backward chunks),
     # used for profiler captures that must stay small on the device.
-    "profile_4k": Workload(
-        name="profile_4k", N=4096, H=4096, V=32768, batch_shape=(1, 4096), w_std=0.02,
-        labels="zipf1.1", ignore_rule="count", ignore_count=204, softcap=0.0,
+    "profile_8k": Workload(
+        name="profile_8k", N=8192, H=4096, V=32768, batch_shape=(1, 8192), w_std=0.02,
+        labels="zipf1.1", ignore_rule="count", ignore_count=409, softcap=0.0,
         reduction="sum", seed=6,
-        description="N=4096 H=4096 V=32768, Zipf(1.1) labels, 5% ignored, sum (profiling size)"),
+        description="N=8192 H=4096 V=32768, Zipf(1.1) labels, 5% ignored, sum (profiling size)"),
 }
 
 # The order of the five problems as they are listed for this workload family.

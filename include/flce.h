@@ -58,8 +58,9 @@
  *  - Return value: argument and launch errors are reported synchronously.
  *    Errors found by the kernels (a label outside [0, V) that is not
  *    ignore_index, a pipeline wait that ran out of time) are recorded in a
- *    status word inside the workspace; flce_get_status() synchronises the
- *    stream and returns them.  Nothing aborts or traps.
+ *    status word inside the workspace.  flce_forward and flce_backward clear
+ *    it first, so flce_get_status() (which synchronises the stream) returns
+ *    the errors of the latest call on that workspace.  Nothing aborts or traps.
  */
 #ifndef FLCE_H
 #define FLCE_H
@@ -118,7 +119,9 @@ flce_status flce_forward(const void* hidden, const void* weight, const int64_t* 
  * Accumulating into d_weight across the micro-batches of one optimizer step
  * (each with grad_scale = 1 / the step's total non-ignored count) gives the
  * token-weighted gradient of the whole batch (modelscope/twinkle PR #335,
- * item 2). */
+ * item 2).  The call clears the workspace status word and records in it a
+ * label outside [0, V) that is not ignore_index (FLCE_ERR_LABEL_RANGE; such a
+ * row contributes only its softmax term, as in the forward). */
 flce_status flce_backward(const void* hidden, const void* weight, const int64_t* labels,
                           const float* lse, int64_t N, int64_t H, int64_t V,
                           int64_t ignore_index, float softcap, int32_t reduction, int32_t dtype,

@@ -31,8 +31,12 @@
 namespace flce {
 namespace {
 
-constexpr int kChunkTokens = 4096;  // multiple of BM
-constexpr int kChunkVocab = 8192;   // multiple of BN
+// Backward chunk: kChunkTokens x kChunkVocab (dZ block 256 MiB bf16).  Longer
+// tiles along the reduced dimensions (K = 16384 for dHidden, 8192 for
+// dWeight) and fewer fp32 read-add-write passes over dHidden and dWeight
+// measured faster than an L2-sized 4096 x 8192 block.
+constexpr int kChunkTokens = 8192;
+constexpr int kChunkVocab = 16384;
 constexpr int kGroupM = 16;
 constexpr size_t kHeaderBytes = 256;
 constexpr int64_t kMaxDim = (int64_t{1} << 31) - 1024;
@@ -178,10 +182,23 @@ struct Chunking {
   int tc, vc;  // chunk sizes (tokens, vocab)
 };
 
+// FLCE_CHUNK_TOKENS / FLCE_CHUNK_VOCAB override the chunk sizes (rounded up to
+// a multiple of 256; read at every call, so flce_workspace_bytes and the
+// calls that use the workspace must see the same values).
+int64_t chunk_size(const char* env, int64_t dflt) {
+  const char* s = std::getenv(env);
+  if (s == nullptr) return dflt;
+  const long long v = std::atoll(s);
+  if (v <= 0) return dflt;
+  return align_up(std::min<int64_t>(v, int64_t{1} << 20), 256);
+}
+
 Chunking chunking(int64_t N, int64_t V) {
   Chunking c;
-  c.tc = static_cast<int>(std::min<int64_t>(kChunkTokens, align_up(std::max<int64_t>(N, 1), BM)));
-  c.vc = static_cast<int>(std::min<int64_t>(kChunkVocab, align_up(V, BN)));
+  const int64_t kt = chunk_size("FLCE_CHUNK_TOKENS", kChunkTokens);
+  const int64_t kv = chunk_size("FLCE_CHUNK_VOCAB", kChunkVocab);
+  c.tc = static_cast<int>(std::min<int64_t>(kt, align_up(std::max<int64_t>(N, 1), BM)));
+  c.vc = static_cast<int>(std::min<int64_t>(kv, align_up(V, BN)));
   return c;
 }
 
@@ -256,6 +273,38 @@ long long* ws_nvalid(void* ws) {
 int cta_group() {
   const char* s = std::getenv("FLCE_CTA_GROUP");
   return (s != nullptr && std::atoi(s) == 1) ? 1 : 2;
+}
+
+// L2 eviction priorities of the GEMM operands and outputs (read at every
+// call; FLCE_L2_HINTS=0 leaves every access at normal priority).
+enum HintUse { kHintFwd, kHintDz, kHintDh, kHintDw };
+void set_l2_hints(GemmArgs& g, HintUse use) {
+  const char* s = std::getenv("FLCE_L2_HINTS");
+  const int preset = s != nullptr ? std::atoi(s) : 1;
+  g.hint_a = g.hint_b = g.hint_out = kL2Normal;
+  if (preset == 0) return;
+  const int hc = preset == 2 ? kL2Normal : kL2Last;  // the token chunk's hidden rows
+  switch (use) {
+    case kHintFwd:
+      g.hint_a = hc;          // hidden: re-read by every vocab tile of its row group
+      g.hint_b = kL2First;    // weight: streamed
+      break;
+    case kHintDz:
+      g.hint_a = hc;          // chunk hidden: re-read by every vocab chunk
+      g.hint_b = preset == 3 ? kL2Last : kL2Normal;  // weight chunk: re-read by dHidden
+      g.hint_out = kL2Last;   // dZ block: read by dHidden and dWeight next
+      break;
+    case kHintDh:
+      g.hint_a = kL2Last;     // dZ block: dWeight reads it too
+      g.hint_b = kL2First;    // weight chunk: last use for this token chunk
+      g.hint_out = kL2First;  // dHidden rows: next touched by the next vocab chunk
+      break;
+    case kHintDw:
+      g.hint_a = kL2First;    // dZ block: last use
+      g.hint_b = hc;          // chunk hidden
+      g.hint_out = kL2First;  // dWeight rows: next touched by the next token chunk
+      break;
+  }
 }
 
 // Backward row compaction: token rows whose label is ignore_index are left out
@@ -429,6 +478,7 @@ flce_status forward_bf16(DevInfo* d, const void* hidden, const void* weight,
   g.b_off = 0;
   g.status = ws_status(ws);
   g.timeout_ns = timeout_ns();
+  set_l2_hints(g, kHintFwd);
 
   cudaError_t e;
   const GemmProblem prob{&ta, &tb, &ta, N, g};
@@ -545,7 +595,8 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
     const int n = static_cast<int>(N);
     const int nblk = (n + kCompactThreads - 1) / kCompactThreads;
     cudaError_t e = launch(kHelper, st, [&] {
-      compact_count_kernel<<<nblk, kCompactThreads, 0, st>>>(labels, n, ignore_index, block_valid);
+      compact_count_kernel<<<nblk, kCompactThreads, 0, st>>>(labels, n, ignore_index, V,
+                                                             ws_status(ws), block_valid);
     });
     if (e == cudaSuccess)
       e = launch(kHelper, st, [&] {
@@ -649,6 +700,7 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
       // dZ overwrites the block the previous chunk's dHidden/dWeight GEMMs read:
       // its main loop may start early, its first store waits for them
       gz.dep_wait = (t0 > 0 || v0 > 0) ? kDepBeforeStores : kDepNone;
+      set_l2_hints(gz, kHintDz);
       cudaError_t e;
       const GemmProblem pz{&t_hid_k, &t_w_k, &t_g_store, rows, gz};
       if (softcap > 0.f) {
@@ -678,6 +730,7 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
       gh.rows_host = rows;
       gh.rows_dim = kRowsM;
       gh.dep_wait = kDepBeforeLoads;  // reads the dZ block written just before
+      set_l2_hints(gh, kHintDh);
       // the last vocab chunk's dHidden epilogue also adds the exact label term
       const bool last_v = v0 + ck.vc >= V;
       StoreEpi::Params eh{static_cast<int>(t0), (v0 > 0 || acc_dh) ? 1 : 0, static_cast<int>(H),
@@ -702,6 +755,7 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
       gw.rows_dim = kRowsK;
       gw.zero_if_empty = (t0 == 0 && !acc_dw) ? 1 : 0;  // the first chunk overwrites dWeight
       gw.dep_wait = kDepBeforeLoads;
+      set_l2_hints(gw, kHintDw);
       StoreEpi::Params ew{static_cast<int>(v0), (t0 > 0 || acc_dw) ? 1 : 0, static_cast<int>(H),
                           static_cast<int>(V), grad_output, grad_scale, n_valid, mean,
                           nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0};
@@ -834,11 +888,19 @@ flce_status flce_backward(const void* hidden, const void* weight, const int64_t*
   s = device_info(&d);
   if (s != FLCE_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e;
+  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(unsigned int), st);  // status word
+  if (e != cudaSuccess) return cuda_fail(e);
   if (N == 0) {
     if (flags & FLCE_ACCUMULATE_DWEIGHT) return FLCE_OK;  // adds nothing
     e = cudaMemsetAsync(d_weight, 0, static_cast<size_t>(V) * H * sizeof(float), st);
     return e == cudaSuccess ? FLCE_OK : cuda_fail(e);
+  }
+  if (!(dtype == FLCE_BF16 && bwd_compact())) {  // the compaction checks the labels itself
+    e = launch(kHelper, st, [&] {
+      label_range_kernel<<<static_cast<unsigned>((N + 255) / 256), 256, 0, st>>>(
+          labels, static_cast<int>(N), ignore_index, V, ws_status(workspace));
+    });
+    if (e != cudaSuccess) return cuda_fail(e);
   }
   const long long* nv = reinterpret_cast<const long long*>(num_valid);
   const bool own_count = (nv == nullptr);

@@ -149,6 +149,17 @@ __global__ void __launch_bounds__(kFinalThreads)
   if (t == 0) *n_valid_out = sc[0];
 }
 
+// Records a label outside [0, V) that is not ignore_index (backward paths that
+// do not compact the rows).
+__global__ void __launch_bounds__(256)
+    label_range_kernel(const int64_t* __restrict__ labels, int N, int64_t ignore_index, int64_t V,
+                       unsigned int* __restrict__ status) {
+  const int i = blockIdx.x * 256 + threadIdx.x;
+  if (i >= N) return;
+  const int64_t y = labels[i];
+  if (y != ignore_index && (y < 0 || y >= V)) atomicOr(status, kStatusLabelRange);
+}
+
 // ------------------------------------------------------------------ row compaction
 // The backward skips token rows whose label is ignore_index (their gradient is
 // exactly zero).  A stable compaction puts the valid rows first, in order, then
@@ -158,10 +169,13 @@ constexpr int kCompactThreads = 1024;
 // Valid rows per block of kCompactThreads rows.
 __global__ void __launch_bounds__(kCompactThreads)
     compact_count_kernel(const int64_t* __restrict__ labels, int N, int64_t ignore_index,
+                         int64_t V, unsigned int* __restrict__ status,
                          int* __restrict__ block_valid) {
   __shared__ int warp_sum[kCompactThreads / 32];
   const int i = blockIdx.x * kCompactThreads + threadIdx.x;
-  const bool v = (i < N) && (labels[i] != ignore_index);
+  const int64_t y = (i < N) ? labels[i] : ignore_index;
+  const bool v = (i < N) && (y != ignore_index);
+  if (v && (y < 0 || y >= V)) atomicOr(status, kStatusLabelRange);
   const unsigned m = __ballot_sync(0xffffffffu, v);
   if ((threadIdx.x & 31) == 0) warp_sum[threadIdx.x >> 5] = __popc(m);
   __syncthreads();

@@ -94,6 +94,9 @@ struct GemmArgs {
   int rows_host;
   int rows_dim;
   int zero_if_empty;
+  // L2 eviction priority (kL2Normal, kL2First, kL2Last) of the A and B operand
+  // loads and of the output stores
+  int hint_a, hint_b, hint_out;
 };
 
 constexpr int kRowsNone = 0;
@@ -227,7 +230,7 @@ struct DzEpi {
     float* resid;  // [token rows] or null
   };
 
-  __device__ static void tile(const Params& p, const GemmArgs&, int m_base, int nb,
+  __device__ static void tile(const Params& p, const GemmArgs& ga, int m_base, int nb,
                               uint32_t taddr, int q, int lane, uint8_t* stg,
                               const CUtensorMap* out, uint32_t tempty, int& nstore, bool) {
     // 64-column chunks whose store box starts inside the block (warp-uniform)
@@ -290,7 +293,8 @@ struct DzEpi {
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        tma_store_2d(out, stg_u32 + b * kStagingBuf, nb * BN + c2 * 64, y0);
+        tma_store_2d_hint(out, stg_u32 + b * kStagingBuf, nb * BN + c2 * 64, y0,
+                          l2_policy(ga.hint_out));
         bulk_commit_group();
       }
       ++nstore;
@@ -336,7 +340,7 @@ struct StoreEpi {
     return g;
   }
 
-  __device__ static void tile(const Params& p, const GemmArgs&, int m_base, int nb,
+  __device__ static void tile(const Params& p, const GemmArgs& ga, int m_base, int nb,
                               uint32_t taddr, int q, int lane, uint8_t* stg,
                               const CUtensorMap* out, uint32_t tempty, int& nstore,
                               bool empty) {
@@ -351,6 +355,7 @@ struct StoreEpi {
       return;
     }
     const float g = empty ? 0.0f : grad_factor(p);  // an empty K range contributes zeros
+    const uint64_t pol = l2_policy(ga.hint_out);
     if (p.row_map != nullptr) {
       const int r = y + lane;
       const bool live = r < y_end;
@@ -387,13 +392,13 @@ struct StoreEpi {
               o.w = fmaf(cfix, w23.y, o.w);
             }
             if (p.reduce) {
-              const float4 a = *d4;
+              const float4 a = ld_f4_hint(d4, pol);
               o.x += a.x;
               o.y += a.y;
               o.z += a.z;
               o.w += a.w;
             }
-            *d4 = o;
+            st_f4_hint(d4, o, pol);
           }
         }
       }
@@ -417,9 +422,9 @@ struct StoreEpi {
       if (lane == 0) {
         const int x = nb * BN + c * 32;
         if (p.reduce)
-          tma_reduce_add_2d(out, stg_u32 + b * kStagingBuf, x, y);
+          tma_reduce_add_2d_hint(out, stg_u32 + b * kStagingBuf, x, y, pol);
         else
-          tma_store_2d(out, stg_u32 + b * kStagingBuf, x, y);
+          tma_store_2d_hint(out, stg_u32 + b * kStagingBuf, x, y, pol);
         bulk_commit_group();
       }
       ++nstore;
@@ -435,11 +440,11 @@ __device__ __forceinline__ void record_timeout(const GemmArgs& g, volatile int* 
 
 template <int kCG>
 __device__ __forceinline__ void load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                        int32_t x, int32_t y) {
+                                        int32_t x, int32_t y, uint64_t policy) {
   if constexpr (kCG == 1)
-    tma_load_2d(dst, map, bar, x, y);
+    tma_load_2d_hint(dst, map, bar, x, y, policy);
   else
-    tma_load_2d_pair(dst, map, bar, x, y);
+    tma_load_2d_pair_hint(dst, map, bar, x, y, policy);
 }
 
 // One launch runs the tiles of one GEMM, or of two independent GEMMs that
@@ -553,7 +558,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // publishes it in a ring slot of both CTAs; every other role reads the
   // same sequence from its own CTA's ring.  A value >= num_tiles ends it.
   auto ring_publish = [&](int slot, uint32_t rph, int t) -> bool {
-    if (!mbar_wait(smem_u32(&ring_empty[slot]), rph ^ 1u, abort_flag, g0.timeout_ns)) return false;
+    // the peer's consumers release the slot remotely: acquire at cluster scope
+    const bool free = (kCG == 2)
+        ? mbar_wait_cluster(smem_u32(&ring_empty[slot]), rph ^ 1u, abort_flag, g0.timeout_ns)
+        : mbar_wait(smem_u32(&ring_empty[slot]), rph ^ 1u, abort_flag, g0.timeout_ns);
+    if (!free) return false;
     tile_ring[slot] = t;
     if constexpr (kCG == 2) {
       const uint32_t peer_slot = mapa_shared(smem_u32(&tile_ring[slot]), 1);
@@ -565,18 +574,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
   // Read the next tile index (all lanes of the calling warp, or one thread).
   auto ring_take = [&](int slot, uint32_t rph, bool warp_wide, int& t) -> bool {
-    bool w = mbar_wait(smem_u32(&ring_full[slot]), rph, abort_flag, g0.timeout_ns);
+    // the peer's copy is written remotely: acquire at cluster scope
+    bool w = (kCG == 2) ? mbar_wait_cluster(smem_u32(&ring_full[slot]), rph, abort_flag,
+                                            g0.timeout_ns)
+                        : mbar_wait(smem_u32(&ring_full[slot]), rph, abort_flag, g0.timeout_ns);
     if (warp_wide) w = __all_sync(0xffffffffu, w);
     if (!w) return false;
-    if constexpr (kCG == 2) fence_acq_rel_cluster();  // the peer's copy is written remotely
     t = *reinterpret_cast<volatile int*>(&tile_ring[slot]);
     if (warp_wide) __syncwarp();
     if (!warp_wide || lane == 0) {
       const uint32_t e = smem_u32(&ring_empty[slot]);
-      if constexpr (kCG == 1)
+      if (kCG == 1 || leader)
         mbar_arrive(e);
       else
-        mbar_arrive_cluster(mapa_shared(e, 0));
+        mbar_arrive_cluster(mapa_shared(e, 0));  // the leader's slot
     }
     return true;
   };
@@ -585,6 +596,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // ---------------- TMA producer (every CTA loads its own halves)
       if (g0.dep_wait == kDepBeforeLoads) griddep_wait();
+      const uint64_t pol_a0 = l2_policy(a0.hint_a), pol_b0 = l2_policy(a0.hint_b);
+      const uint64_t pol_a1 = l2_policy(a1.hint_a), pol_b1 = l2_policy(a1.hint_b);
       uint32_t stage = 0, phase = 0;
       uint32_t issued_mask = 0, issued_par = 0;
       bool ok = true;
@@ -611,6 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const CUtensorMap* mB = prob ? &tmB1 : &tmB0;
         const bool a_mn = prob ? kAMn1 : kAMn0;
         const bool b_mn = prob ? kBMn1 : kBMn0;
+        const uint64_t pol_a = prob ? pol_a1 : pol_a0, pol_b = prob ? pol_b1 : pol_b0;
         const int m_cta = mb * Cfg::kUnitRows + static_cast<int>(rank) * BM;
         const int n_cta = nb * BN + static_cast<int>(rank) * Cfg::kBRows;
         for (int kb = 0; kb < g.k_blocks; ++kb) {
@@ -632,16 +646,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (a_mn) {
 #pragma unroll
             for (int c = 0; c < BM / 64; ++c)
-              load_2d<kCG>(sa + c * 8192, mA, fb, m_cta + c * 64, g.a_off + kb * BK);
+              load_2d<kCG>(sa + c * 8192, mA, fb, m_cta + c * 64, g.a_off + kb * BK, pol_a);
           } else {
-            load_2d<kCG>(sa, mA, fb, kb * BK, g.a_off + m_cta);
+            load_2d<kCG>(sa, mA, fb, kb * BK, g.a_off + m_cta, pol_a);
           }
           if (b_mn) {
 #pragma unroll
             for (int c = 0; c < Cfg::kBRows / 64; ++c)
-              load_2d<kCG>(sb + c * 8192, mB, fb, n_cta + c * 64, g.b_off + kb * BK);
+              load_2d<kCG>(sb + c * 8192, mB, fb, n_cta + c * 64, g.b_off + kb * BK, pol_b);
           } else {
-            load_2d<kCG>(sb, mB, fb, kb * BK, g.b_off + n_cta);
+            load_2d<kCG>(sb, mB, fb, kb * BK, g.b_off + n_cta, pol_b);
           }
           issued_mask |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);

@@ -12,6 +12,9 @@ Tolerances come from the contract of this FLCE build:
                                   wide margin while still catching any
                                   dropped tile or wrong column (>= 1e-2).
 """
+import contextlib
+import os
+
 import numpy as np
 import torch
 
@@ -53,3 +56,23 @@ def small_inputs(N, H, V, seed, n_ign, w_std=0.05):
     """Seeded ad-hoc problem with the workload recipe (bf16-quantised)."""
     w = fi.custom_workload(N, H, V, seed=seed, w_std=w_std, ignore_count=n_ign)
     return fi.make_inputs(w, keep_raw=True)
+
+
+@contextlib.contextmanager
+def chunks(tokens: int, vocab: int):
+    """Run the backward with tokens x vocab chunks instead of the default
+    8192 x 16384, so that small problems span several chunks along both
+    reduced dimensions (FLCE_CHUNK_TOKENS / FLCE_CHUNK_VOCAB, read by the
+    library at every call)."""
+    keys = ("FLCE_CHUNK_TOKENS", "FLCE_CHUNK_VOCAB")
+    old = {k: os.environ.get(k) for k in keys}
+    os.environ["FLCE_CHUNK_TOKENS"] = str(tokens)
+    os.environ["FLCE_CHUNK_VOCAB"] = str(vocab)
+    try:
+        yield
+    finally:
+        for k, v in old.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v

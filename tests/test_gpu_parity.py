@@ -1,6 +1,9 @@
 """GPU parity of the CUDA path (through the C ABI) against the float64 oracle
 on small problems that span several tiles, ragged tails and several backward
 chunks, plus the edge cases of the method."""
+import contextlib
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -72,12 +75,19 @@ def test_ragged_multi_tile(softcap, reduction):
             grad_output=0.75)
 
 
+SMALL_CHUNKS = (1024, 2048)  # tokens x vocab per backward chunk in the multi-chunk tests
+
+
+@pytest.mark.parametrize("chunked", [False, True])
 @pytest.mark.parametrize("softcap", [0.0, 3.0])
-def test_several_backward_chunks(softcap):
-    # 2 token chunks x 2 vocab chunks: exercises the TMA reduce-add accumulation
+def test_several_backward_chunks(softcap, chunked):
+    # default chunks: one chunk; 1024 x 2048 chunks: 5 token x 5 vocab chunks, which
+    # exercises the cross-chunk accumulation (dWeight TMA reduce-add, dHidden
+    # read-add-write) and the ragged last chunk of each dimension
     inp = G.small_inputs(N=4500, H=136, V=9000, seed=8, n_ign=450, w_std=0.1)
-    got = run(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
-              G.labels_tensor(inp.labels), softcap, "sum", grad_scale=1.0 / 4050)
+    with G.chunks(*SMALL_CHUNKS) if chunked else contextlib.nullcontext():
+        got = run(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
+                  G.labels_tensor(inp.labels), softcap, "sum", grad_scale=1.0 / 4050)
     compare(got, inp.hidden, inp.weight, inp.labels, softcap, "sum", grad_scale=1.0 / 4050)
 
 
@@ -124,9 +134,27 @@ def test_label_out_of_range_is_reported():
         flce.forward(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
                      G.labels_tensor(y), check_status=True)
     assert e.value.status == 3
-    # the status is cleared by the next forward
-    flce.forward(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
-                 G.labels_tensor(inp.labels), check_status=True)
+    # the backward finds the same label on its own (compacted bf16, uncompacted, fp32)
+    h, W = G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits)
+    lse = torch.zeros(130, device="cuda")
+    for env in ("1", "0"):
+        os.environ["FLCE_BWD_COMPACT"] = env
+        try:
+            with pytest.raises(flce.FlceError) as e:
+                flce.backward(h, W, G.labels_tensor(y), lse, check_status=True)
+            assert e.value.status == 3
+        finally:
+            os.environ.pop("FLCE_BWD_COMPACT", None)
+    with pytest.raises(flce.FlceError) as e:
+        flce.backward(G.f32_tensor(inp.hidden_raw), G.f32_tensor(inp.weight_raw),
+                      G.labels_tensor(y), lse, check_status=True)
+    assert e.value.status == 3
+    # the status is cleared by the next forward ...
+    f = flce.forward(h, W, G.labels_tensor(inp.labels), check_status=True)
+    # ... and by the next backward, also on a workspace never used before
+    ws = flce.alloc_workspace(130, 64, 300, torch.bfloat16, "cuda")
+    ws.fill_(255)
+    flce.backward(h, W, G.labels_tensor(inp.labels), f.lse, workspace=ws, check_status=True)
 
 
 def test_module_autograd_and_num_tokens_contract():
@@ -152,8 +180,9 @@ def test_repeated_calls_are_deterministic():
     inp = G.small_inputs(N=4200, H=128, V=8500, seed=14, n_ign=100)
     args = (G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
             G.labels_tensor(inp.labels), 0.0, "sum")
-    a = run(*args)
-    b = run(*args)
+    with G.chunks(*SMALL_CHUNKS):
+        a = run(*args)
+        b = run(*args)
     assert a["loss"] == b["loss"]
     assert np.array_equal(a["lse"], b["lse"])
     assert np.array_equal(a["dh"], b["dh"]) and np.array_equal(a["dw"], b["dw"])
@@ -168,19 +197,20 @@ def test_accumulate_flags(dtype):
         inp = G.small_inputs(N=96, H=64, V=700, seed=15, n_ign=10, w_std=0.1)
         h, W = G.f32_tensor(inp.hidden_raw), G.f32_tensor(inp.weight_raw)
     y = G.labels_tensor(inp.labels)
-    f = flce.forward(h, W, y, check_status=True)
-    dh1, dw1 = flce.backward(h, W, y, f.lse, grad_scale=0.5, check_status=True)
-    dh2, dw2 = dh1.clone(), dw1.clone()
-    flce.backward(h, W, y, f.lse, grad_scale=0.5, d_hidden=dh2, d_weight=dw2,
-                  accumulate_d_hidden=True, accumulate_d_weight=True, check_status=True)
-    torch.cuda.synchronize()
-    assert G.rel_l2(dh2.cpu().numpy(), 2 * dh1.cpu().numpy().astype(np.float64)) <= 1e-6
-    assert G.rel_l2(dw2.cpu().numpy(), 2 * dw1.cpu().numpy().astype(np.float64)) <= 1e-6
-    # accumulate only dWeight: dHidden is overwritten
-    dh3, dw3 = dh1.clone(), dw1.clone()
-    flce.backward(h, W, y, f.lse, grad_scale=0.5, d_hidden=dh3, d_weight=dw3,
-                  accumulate_d_weight=True, check_status=True)
-    assert torch.equal(dh3, dh1)
+    with G.chunks(*SMALL_CHUNKS):
+        f = flce.forward(h, W, y, check_status=True)
+        dh1, dw1 = flce.backward(h, W, y, f.lse, grad_scale=0.5, check_status=True)
+        dh2, dw2 = dh1.clone(), dw1.clone()
+        flce.backward(h, W, y, f.lse, grad_scale=0.5, d_hidden=dh2, d_weight=dw2,
+                      accumulate_d_hidden=True, accumulate_d_weight=True, check_status=True)
+        torch.cuda.synchronize()
+        assert G.rel_l2(dh2.cpu().numpy(), 2 * dh1.cpu().numpy().astype(np.float64)) <= 1e-6
+        assert G.rel_l2(dw2.cpu().numpy(), 2 * dw1.cpu().numpy().astype(np.float64)) <= 1e-6
+        # accumulate only dWeight: dHidden is overwritten
+        dh3, dw3 = dh1.clone(), dw1.clone()
+        flce.backward(h, W, y, f.lse, grad_scale=0.5, d_hidden=dh3, d_weight=dw3,
+                      accumulate_d_weight=True, check_status=True)
+        assert torch.equal(dh3, dh1)
 
 
 def test_microbatch_accumulation_matches_full_batch():
@@ -188,15 +218,16 @@ def test_microbatch_accumulation_matches_full_batch():
     h, W, y = (G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
                G.labels_tensor(inp.labels))
     n = int((inp.labels != IGN).sum())
-    f = flce.forward(h, W, y)
-    dh_full, dw_full = flce.backward(h, W, y, f.lse, grad_scale=1.0 / n)
-    dw_acc = torch.empty_like(dw_full)
-    dh_acc = torch.empty_like(dh_full)
-    for k, sl in enumerate([slice(0, 1500), slice(1500, 4400)]):
-        fk = flce.forward(h[sl], W, y[sl], check_status=True)
-        flce.backward(h[sl], W, y[sl], fk.lse, grad_scale=1.0 / n, d_hidden=dh_acc[sl],
-                      d_weight=dw_acc, accumulate_d_weight=(k > 0), check_status=True)
-    torch.cuda.synchronize()
+    with G.chunks(*SMALL_CHUNKS):
+        f = flce.forward(h, W, y)
+        dh_full, dw_full = flce.backward(h, W, y, f.lse, grad_scale=1.0 / n)
+        dw_acc = torch.empty_like(dw_full)
+        dh_acc = torch.empty_like(dh_full)
+        for k, sl in enumerate([slice(0, 1500), slice(1500, 4400)]):
+            fk = flce.forward(h[sl], W, y[sl], check_status=True)
+            flce.backward(h[sl], W, y[sl], fk.lse, grad_scale=1.0 / n, d_hidden=dh_acc[sl],
+                          d_weight=dw_acc, accumulate_d_weight=(k > 0), check_status=True)
+        torch.cuda.synchronize()
     assert G.rel_l2(dw_acc.cpu().numpy(), dw_full.cpu().numpy().astype(np.float64)) <= 1e-5
     assert G.rel_l2(dh_acc.cpu().numpy(), dh_full.cpu().numpy().astype(np.float64)) <= 1e-6
 
@@ -228,9 +259,11 @@ def test_label_term_is_exact(case):
     inp, softcap, red, gs = _label_term_case(case)
     args = (G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
             G.labels_tensor(inp.labels), softcap, red)
-    got = run(*args, grad_scale=gs)
+    with G.chunks(*SMALL_CHUNKS) if case in ("softcap_chunks", "zipf_runs") else \
+            contextlib.nullcontext():
+        got = run(*args, grad_scale=gs)
+        again = run(*args, grad_scale=gs)  # the per-label sums have a fixed order
     rb = oracle.backward(inp.hidden, inp.weight, inp.labels, IGN, softcap, red, grad_scale=gs)
     assert G.rel_l2(got["dh"], rb["d_hidden"]) <= 4e-4
     assert G.rel_l2(got["dw"], rb["d_weight"]) <= 4e-4
-    again = run(*args, grad_scale=gs)  # the per-label sums have a fixed order
     assert np.array_equal(got["dh"], again["dh"]) and np.array_equal(got["dw"], again["dw"])
