@@ -37,7 +37,10 @@ namespace {
 // measured faster than an L2-sized 4096 x 8192 block.
 constexpr int kChunkTokens = 8192;
 constexpr int kChunkVocab = 16384;
-constexpr int kGroupM = 16;
+constexpr int kGroupM = 16;     // forward and dZ
+constexpr int kGroupMGrad = 8;  // dHidden and dWeight: their long-K panels (8 MiB at the bench
+                                // size) make a 16-tile group's panels overflow L2 (ncu: 2.4 vs
+                                // 2.8 GB of DRAM reads per launch)
 constexpr size_t kHeaderBytes = 256;
 constexpr int64_t kMaxDim = (int64_t{1} << 31) - 1024;
 constexpr int kSimtMaxH = 12288;
@@ -148,6 +151,24 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// The 3-D chunk view of a row-major bf16 matrix [k_rows, mn] (row pitch
+// row_bytes) for MN-major operand loads: x = 64 elements within a chunk, y =
+// row, z = 64-element chunk, box {64, BK, 2}.  mn must be a multiple of 64 and
+// every chunk must lie inside the allocation (x is not clipped per row).
+bool make_map_mn3d(CUtensorMap* m, const void* base, uint64_t mn, uint64_t k_rows,
+                   uint64_t row_bytes) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr || mn % 64 != 0) return false;
+  cuuint64_t dims[3] = {64, k_rows, mn / 64};
+  cuuint64_t strides[2] = {row_bytes, 128};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(BK), 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -273,37 +294,6 @@ long long* ws_nvalid(void* ws) {
 int cta_group() {
   const char* s = std::getenv("FLCE_CTA_GROUP");
   return (s != nullptr && std::atoi(s) == 1) ? 1 : 2;
-}
-
-// L2 eviction priorities of the GEMM operands and outputs (read at every
-// call; FLCE_L2_HINTS=0 leaves every access at normal priority).  Measured
-// neutral at the bench size (within the power-capped clock's noise); kept
-// because they state each access's reuse.
-enum HintUse { kHintFwd, kHintDz, kHintDh, kHintDw };
-void set_l2_hints(GemmArgs& g, HintUse use) {
-  g.hint_a = g.hint_b = g.hint_out = kL2Normal;
-  const char* s = std::getenv("FLCE_L2_HINTS");
-  if (s != nullptr && std::atoi(s) == 0) return;
-  switch (use) {
-    case kHintFwd:
-      g.hint_a = kL2Last;     // hidden: re-read by every vocab tile of its row group
-      g.hint_b = kL2First;    // weight: streamed
-      break;
-    case kHintDz:
-      g.hint_a = kL2Last;     // chunk hidden: re-read by every vocab chunk
-      g.hint_out = kL2Last;   // dZ block: read by dHidden and dWeight next
-      break;
-    case kHintDh:
-      g.hint_a = kL2Last;     // dZ block: dWeight reads it too
-      g.hint_b = kL2First;    // weight chunk: last use for this token chunk
-      g.hint_out = kL2First;  // dHidden rows: next touched by the next vocab chunk
-      break;
-    case kHintDw:
-      g.hint_a = kL2First;    // dZ block: last use
-      g.hint_b = kL2Last;     // chunk hidden
-      g.hint_out = kL2First;  // dWeight rows: next touched by the next token chunk
-      break;
-  }
 }
 
 // Backward row compaction: token rows whose label is ignore_index are left out
@@ -477,7 +467,6 @@ flce_status forward_bf16(DevInfo* d, const void* hidden, const void* weight,
   g.b_off = 0;
   g.status = ws_status(ws);
   g.timeout_ns = timeout_ns();
-  set_l2_hints(g, kHintFwd);
 
   cudaError_t e;
   const GemmProblem prob{&ta, &tb, &ta, N, g};
@@ -662,6 +651,14 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
       !make_map(&t_dh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d_hidden, H, N, H * 4, 32, 32) ||
       !make_map(&t_dw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d_weight, H, V, H * 4, 32, 32))
     return FLCE_ERR_CUDA;
+  // H a multiple of 64: the MN-major hidden and weight operands use the 3-D view
+  // (FLCE_MN3D=0: every MN-major operand uses the 2-D view; read at every call)
+  const char* mn3d_env = std::getenv("FLCE_MN3D");
+  const bool mn3d = !(mn3d_env != nullptr && std::atoi(mn3d_env) == 0);
+  const bool h3d = mn3d && (H % 64 == 0);
+  if (h3d && (!make_map_mn3d(&t_hid_mn, hid, H, N, H * 2) ||
+              !make_map_mn3d(&t_w_mn, weight, H, V, H * 2)))
+    return FLCE_ERR_CUDA;
 
   const int n_tiles_h = static_cast<int>((H + BN - 1) / BN);
   const int k_blocks_h = static_cast<int>((H + BK - 1) / BK);
@@ -678,9 +675,13 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
                     static_cast<uint64_t>(ck.vc) * 2, 64, 32) ||
           !make_map(&t_g_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, gbuf, cols, rows,
                     static_cast<uint64_t>(ck.vc) * 2, BK, BM) ||
-          !make_map(&t_g_mn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, gbuf, cols, rows,
-                    static_cast<uint64_t>(ck.vc) * 2, 64, BK))
+          !(mn3d ? make_map_mn3d(&t_g_mn, gbuf, ck.vc, rows, static_cast<uint64_t>(ck.vc) * 2)
+                 : make_map(&t_g_mn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, gbuf, cols, rows,
+                            static_cast<uint64_t>(ck.vc) * 2, 64, BK)))
         return FLCE_ERR_CUDA;
+      // (the dZ block's 3-D view spans its full row pitch: columns past `cols`
+      // hold stale values that reach only dWeight rows past V, which the
+      // output map clips)
 
       // 1) dZ = f(hidden[t0:] . W[v0:]^T) -> bf16 block
       GemmArgs gz{};
@@ -699,7 +700,6 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
       // dZ overwrites the block the previous chunk's dHidden/dWeight GEMMs read:
       // its main loop may start early, its first store waits for them
       gz.dep_wait = (t0 > 0 || v0 > 0) ? kDepBeforeStores : kDepNone;
-      set_l2_hints(gz, kHintDz);
       cudaError_t e;
       const GemmProblem pz{&t_hid_k, &t_w_k, &t_g_store, rows, gz};
       if (softcap > 0.f) {
@@ -718,7 +718,7 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
       GemmArgs gh{};
       gh.n_tiles = n_tiles_h;
       gh.k_blocks = (cols + BK - 1) / BK;
-      gh.group_m = kGroupM;
+      gh.group_m = kGroupMGrad;
       gh.a_off = 0;
       gh.b_off = static_cast<int>(v0);
       gh.status = ws_status(ws);
@@ -729,7 +729,7 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
       gh.rows_host = rows;
       gh.rows_dim = kRowsM;
       gh.dep_wait = kDepBeforeLoads;  // reads the dZ block written just before
-      set_l2_hints(gh, kHintDh);
+      gh.b_mn3d = h3d ? 1 : 0;
       // the last vocab chunk's dHidden epilogue also adds the exact label term
       const bool last_v = v0 + ck.vc >= V;
       StoreEpi::Params eh{static_cast<int>(t0), (v0 > 0 || acc_dh) ? 1 : 0, static_cast<int>(H),
@@ -742,7 +742,7 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
       GemmArgs gw{};
       gw.n_tiles = n_tiles_h;
       gw.k_blocks = (rows + BK - 1) / BK;
-      gw.group_m = kGroupM;
+      gw.group_m = kGroupMGrad;
       gw.a_off = 0;
       gw.b_off = static_cast<int>(t0);
       gw.status = ws_status(ws);
@@ -754,7 +754,8 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
       gw.rows_dim = kRowsK;
       gw.zero_if_empty = (t0 == 0 && !acc_dw) ? 1 : 0;  // the first chunk overwrites dWeight
       gw.dep_wait = kDepBeforeLoads;
-      set_l2_hints(gw, kHintDw);
+      gw.a_mn3d = mn3d ? 1 : 0;
+      gw.b_mn3d = h3d ? 1 : 0;
       StoreEpi::Params ew{static_cast<int>(v0), (t0 > 0 || acc_dw) ? 1 : 0, static_cast<int>(H),
                           static_cast<int>(V), grad_output, grad_scale, n_valid, mean,
                           nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0};

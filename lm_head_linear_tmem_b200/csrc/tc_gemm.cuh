@@ -94,9 +94,11 @@ struct GemmArgs {
   int rows_host;
   int rows_dim;
   int zero_if_empty;
-  // L2 eviction priority (kL2Normal, kL2First, kL2Last) of the A and B operand
-  // loads and of the output stores
-  int hint_a, hint_b, hint_out;
+  // An MN-major operand whose map is the 3-D chunk view (x = 64 elements of a
+  // 64-wide MN chunk, y = K row, z = chunk; one 16 KiB box = two chunks of 64 K
+  // rows) instead of the 2-D view (one 8 KiB box per chunk).  Fewer, larger
+  // TMA requests: 76.7 vs 68.9 B/clk per SM measured into shared memory.
+  int a_mn3d, b_mn3d;
 };
 
 constexpr int kRowsNone = 0;
@@ -230,7 +232,7 @@ struct DzEpi {
     float* resid;  // [token rows] or null
   };
 
-  __device__ static void tile(const Params& p, const GemmArgs& ga, int m_base, int nb,
+  __device__ static void tile(const Params& p, const GemmArgs&, int m_base, int nb,
                               uint32_t taddr, int q, int lane, uint8_t* stg,
                               const CUtensorMap* out, uint32_t tempty, int& nstore, bool) {
     // 64-column chunks whose store box starts inside the block (warp-uniform)
@@ -293,8 +295,7 @@ struct DzEpi {
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        tma_store_2d_hint(out, stg_u32 + b * kStagingBuf, nb * BN + c2 * 64, y0,
-                          l2_policy(ga.hint_out));
+        tma_store_2d(out, stg_u32 + b * kStagingBuf, nb * BN + c2 * 64, y0);
         bulk_commit_group();
       }
       ++nstore;
@@ -340,7 +341,7 @@ struct StoreEpi {
     return g;
   }
 
-  __device__ static void tile(const Params& p, const GemmArgs& ga, int m_base, int nb,
+  __device__ static void tile(const Params& p, const GemmArgs&, int m_base, int nb,
                               uint32_t taddr, int q, int lane, uint8_t* stg,
                               const CUtensorMap* out, uint32_t tempty, int& nstore,
                               bool empty) {
@@ -355,7 +356,6 @@ struct StoreEpi {
       return;
     }
     const float g = empty ? 0.0f : grad_factor(p);  // an empty K range contributes zeros
-    const uint64_t pol = l2_policy(ga.hint_out);
     if (p.row_map != nullptr) {
       const int r = y + lane;
       const bool live = r < y_end;
@@ -392,13 +392,13 @@ struct StoreEpi {
               o.w = fmaf(cfix, w23.y, o.w);
             }
             if (p.reduce) {
-              const float4 a = ld_f4_hint(d4, pol);
+              const float4 a = *d4;
               o.x += a.x;
               o.y += a.y;
               o.z += a.z;
               o.w += a.w;
             }
-            st_f4_hint(d4, o, pol);
+            *d4 = o;
           }
         }
       }
@@ -422,9 +422,9 @@ struct StoreEpi {
       if (lane == 0) {
         const int x = nb * BN + c * 32;
         if (p.reduce)
-          tma_reduce_add_2d_hint(out, stg_u32 + b * kStagingBuf, x, y, pol);
+          tma_reduce_add_2d(out, stg_u32 + b * kStagingBuf, x, y);
         else
-          tma_store_2d_hint(out, stg_u32 + b * kStagingBuf, x, y, pol);
+          tma_store_2d(out, stg_u32 + b * kStagingBuf, x, y);
         bulk_commit_group();
       }
       ++nstore;
@@ -440,11 +440,28 @@ __device__ __forceinline__ void record_timeout(const GemmArgs& g, volatile int* 
 
 template <int kCG>
 __device__ __forceinline__ void load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                        int32_t x, int32_t y, uint64_t policy) {
+                                        int32_t x, int32_t y) {
   if constexpr (kCG == 1)
-    tma_load_2d_hint(dst, map, bar, x, y, policy);
+    tma_load_2d(dst, map, bar, x, y);
   else
-    tma_load_2d_pair_hint(dst, map, bar, x, y, policy);
+    tma_load_2d_pair(dst, map, bar, x, y);
+}
+
+// An MN-major operand tile of `rows` MN elements x BK K rows starting at MN
+// coordinate mn (a multiple of 128) and K row k: 64-element chunks 8 KiB apart.
+template <int kCG>
+__device__ __forceinline__ void load_mn(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                        int rows, int mn, int k, bool view3d) {
+  if (view3d) {
+    for (int c = 0; c < rows / 128; ++c) {
+      if constexpr (kCG == 1)
+        tma_load_3d(dst + c * 16384, map, bar, 0, k, mn / 64 + 2 * c);
+      else
+        tma_load_3d_pair(dst + c * 16384, map, bar, 0, k, mn / 64 + 2 * c);
+    }
+  } else {
+    for (int c = 0; c < rows / 64; ++c) load_2d<kCG>(dst + c * 8192, map, bar, mn + c * 64, k);
+  }
 }
 
 // One launch runs the tiles of one GEMM, or of two independent GEMMs that
@@ -596,8 +613,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // ---------------- TMA producer (every CTA loads its own halves)
       if (g0.dep_wait == kDepBeforeLoads) griddep_wait();
-      const uint64_t pol_a0 = l2_policy(a0.hint_a), pol_b0 = l2_policy(a0.hint_b);
-      const uint64_t pol_a1 = l2_policy(a1.hint_a), pol_b1 = l2_policy(a1.hint_b);
       uint32_t stage = 0, phase = 0;
       uint32_t issued_mask = 0, issued_par = 0;
       bool ok = true;
@@ -624,7 +639,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const CUtensorMap* mB = prob ? &tmB1 : &tmB0;
         const bool a_mn = prob ? kAMn1 : kAMn0;
         const bool b_mn = prob ? kBMn1 : kBMn0;
-        const uint64_t pol_a = prob ? pol_a1 : pol_a0, pol_b = prob ? pol_b1 : pol_b0;
         const int m_cta = mb * Cfg::kUnitRows + static_cast<int>(rank) * BM;
         const int n_cta = nb * BN + static_cast<int>(rank) * Cfg::kBRows;
         for (int kb = 0; kb < g.k_blocks; ++kb) {
@@ -644,18 +658,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t sa = smem_u32(smem + stage * Cfg::kStageBytes);
           const uint32_t sb = sa + kABytes;
           if (a_mn) {
-#pragma unroll
-            for (int c = 0; c < BM / 64; ++c)
-              load_2d<kCG>(sa + c * 8192, mA, fb, m_cta + c * 64, g.a_off + kb * BK, pol_a);
+            load_mn<kCG>(sa, mA, fb, BM, m_cta, g.a_off + kb * BK, g.a_mn3d != 0);
           } else {
-            load_2d<kCG>(sa, mA, fb, kb * BK, g.a_off + m_cta, pol_a);
+            load_2d<kCG>(sa, mA, fb, kb * BK, g.a_off + m_cta);
           }
           if (b_mn) {
-#pragma unroll
-            for (int c = 0; c < Cfg::kBRows / 64; ++c)
-              load_2d<kCG>(sb + c * 8192, mB, fb, n_cta + c * 64, g.b_off + kb * BK, pol_b);
+            load_mn<kCG>(sb, mB, fb, Cfg::kBRows, n_cta, g.b_off + kb * BK, g.b_mn3d != 0);
           } else {
-            load_2d<kCG>(sb, mB, fb, kb * BK, g.b_off + n_cta, pol_b);
+            load_2d<kCG>(sb, mB, fb, kb * BK, g.b_off + n_cta);
           }
           issued_mask |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
