@@ -91,6 +91,11 @@ typedef enum flce_dtype { FLCE_BF16 = 0, FLCE_FP32 = 1 } flce_dtype;
  * Returns 0 for invalid sizes.  Pure host computation. */
 size_t flce_workspace_bytes(int64_t N, int64_t H, int64_t V, int32_t dtype);
 
+/* The same for a flce_backward call with these flags: FLCE_DHIDDEN_BF16 and
+ * FLCE_DWEIGHT_BF16 add fp32 scratch for the gradient before its single
+ * rounding (4*N*H and 4*V*H bytes).  Returns 0 for invalid sizes or flags. */
+size_t flce_workspace_bytes_ex(int64_t N, int64_t H, int64_t V, int32_t dtype, int32_t flags);
+
 /* Forward.
  *   loss        device float[1]   'sum' or 'mean' loss (float32)
  *   num_tokens  device int64[1]   n for 'sum', 0 for 'mean'
@@ -106,6 +111,8 @@ flce_status flce_forward(const void* hidden, const void* weight, const int64_t* 
 /* flce_backward flags. */
 #define FLCE_ACCUMULATE_DHIDDEN 1 /* d_hidden += gradient (else overwritten) */
 #define FLCE_ACCUMULATE_DWEIGHT 2 /* d_weight += gradient (else overwritten) */
+#define FLCE_DHIDDEN_BF16 4       /* d_hidden is bf16 [N*H] (else float) */
+#define FLCE_DWEIGHT_BF16 8       /* d_weight is bf16 [V*H] (else float) */
 
 /* Backward of the loss returned by flce_forward with the same arguments.
  *   lse          device float[N]  from flce_forward
@@ -114,8 +121,15 @@ flce_status flce_forward(const void* hidden, const void* weight, const int64_t* 
  *   num_valid    device int64[1]  n (the true count, also for 'mean');
  *                                 NULL: the library counts it on the device
  *   d_hidden     device float[N*H]  overwritten, or accumulated into
+ *                (bf16[N*H] with FLCE_DHIDDEN_BF16)
  *   d_weight     device float[V*H]  overwritten, or accumulated into
- *   flags        FLCE_ACCUMULATE_DHIDDEN | FLCE_ACCUMULATE_DWEIGHT, or 0.
+ *                (bf16[V*H] with FLCE_DWEIGHT_BF16)
+ *   flags        any OR of FLCE_ACCUMULATE_DHIDDEN, FLCE_ACCUMULATE_DWEIGHT,
+ *                FLCE_DHIDDEN_BF16, FLCE_DWEIGHT_BF16, or 0.
+ * A bf16 output is computed in fp32 scratch inside the workspace (size it with
+ * flce_workspace_bytes_ex) and rounded once, to nearest even: overwrite gives
+ * bf16(g), accumulate gives bf16(float(old) + g).  Ignored rows of a
+ * non-accumulated d_hidden are exact zeros either way.
  * Accumulating into d_weight across the micro-batches of one optimizer step
  * (each with grad_scale = 1 / the step's total non-ignored count) gives the
  * token-weighted gradient of the whole batch (modelscope/twinkle PR #335,

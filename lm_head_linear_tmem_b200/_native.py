@@ -26,10 +26,12 @@ STATUS_NAMES = {
 SUM, MEAN = 0, 1
 BF16, FP32 = 0, 1
 ACCUMULATE_DHIDDEN, ACCUMULATE_DWEIGHT = 1, 2
+DHIDDEN_BF16, DWEIGHT_BF16 = 4, 8
 
 # Every symbol include/flce.h declares, with its ctypes signature.
 SIGNATURES = {
     "flce_workspace_bytes": (c_size, [c_i64, c_i64, c_i64, c_i32]),
+    "flce_workspace_bytes_ex": (c_size, [c_i64, c_i64, c_i64, c_i32, c_i32]),
     "flce_forward": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32, c_i32,
                              c_i32, c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),
     "flce_backward": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32,

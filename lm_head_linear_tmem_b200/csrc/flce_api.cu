@@ -283,6 +283,26 @@ size_t ws_bytes(int64_t N, int64_t H, int64_t V, bool bf16) {
   return align_up(std::max(fwd_layout(N, V, bf16).end, bwd_bytes(N, H, V, bf16)), 256);
 }
 
+// bf16 gradient outputs: fp32 scratch for dHidden and/or dWeight after the
+// shape's own workspace.
+constexpr int32_t kBf16OutFlags = FLCE_DHIDDEN_BF16 | FLCE_DWEIGHT_BF16;
+constexpr int32_t kAllBwdFlags = FLCE_ACCUMULATE_DHIDDEN | FLCE_ACCUMULATE_DWEIGHT | kBf16OutFlags;
+
+struct GradScratch {
+  size_t dh, dw, end;  // byte offsets (dh / dw meaningful only with their flag)
+};
+
+GradScratch grad_scratch(int64_t N, int64_t H, int64_t V, bool bf16, int32_t flags) {
+  GradScratch g{};
+  size_t off = align_up(ws_bytes(N, H, V, bf16), 256);
+  g.dh = off;
+  if (flags & FLCE_DHIDDEN_BF16) off = align_up(off + 4 * static_cast<size_t>(N) * H, 256);
+  g.dw = off;
+  if (flags & FLCE_DWEIGHT_BF16) off = align_up(off + 4 * static_cast<size_t>(V) * H, 256);
+  g.end = off;
+  return g;
+}
+
 unsigned int* ws_status(void* ws) { return reinterpret_cast<unsigned int*>(ws); }
 long long* ws_nvalid(void* ws) {
   return reinterpret_cast<long long*>(reinterpret_cast<char*>(ws) + 8);
@@ -841,6 +861,12 @@ size_t flce_workspace_bytes(int64_t N, int64_t H, int64_t V, int32_t dtype) {
   return ws_bytes(N, H, V, dtype == FLCE_BF16);
 }
 
+size_t flce_workspace_bytes_ex(int64_t N, int64_t H, int64_t V, int32_t dtype, int32_t flags) {
+  if ((flags & ~kAllBwdFlags) != 0) return 0;
+  if (flce_workspace_bytes(N, H, V, dtype) == 0) return 0;
+  return grad_scratch(N, H, V, dtype == FLCE_BF16, flags).end;
+}
+
 flce_status flce_forward(const void* hidden, const void* weight, const int64_t* labels,
                          int64_t N, int64_t H, int64_t V, int64_t ignore_index, float softcap,
                          int32_t reduction, int32_t dtype, float* loss, int64_t* num_tokens,
@@ -875,10 +901,12 @@ flce_status flce_backward(const void* hidden, const void* weight, const int64_t*
                           const float* grad_output, float grad_scale, const int64_t* num_valid,
                           float* d_hidden, float* d_weight, int32_t flags, void* workspace,
                           size_t workspace_bytes, void* stream) {
-  if ((flags & ~(FLCE_ACCUMULATE_DHIDDEN | FLCE_ACCUMULATE_DWEIGHT)) != 0) return FLCE_ERR_ARG;
+  if ((flags & ~kAllBwdFlags) != 0) return FLCE_ERR_ARG;
   flce_status s = check_common(hidden, weight, labels, N, H, V, softcap, reduction, dtype,
                                workspace, workspace_bytes);
   if (s != FLCE_OK) return s;
+  const GradScratch gs = grad_scratch(N, H, V, dtype == FLCE_BF16, flags);
+  if (workspace_bytes < gs.end) return FLCE_ERR_WORKSPACE;
   if (d_weight == nullptr || (N > 0 && (d_hidden == nullptr || lse == nullptr)))
     return FLCE_ERR_ARG;
   if (!aligned16(d_hidden) || !aligned16(d_weight)) return FLCE_ERR_ARG;
@@ -892,9 +920,18 @@ flce_status flce_backward(const void* hidden, const void* weight, const int64_t*
   if (e != cudaSuccess) return cuda_fail(e);
   if (N == 0) {
     if (flags & FLCE_ACCUMULATE_DWEIGHT) return FLCE_OK;  // adds nothing
-    e = cudaMemsetAsync(d_weight, 0, static_cast<size_t>(V) * H * sizeof(float), st);
+    const size_t elem = (flags & FLCE_DWEIGHT_BF16) ? 2 : sizeof(float);  // +0.0 in both
+    e = cudaMemsetAsync(d_weight, 0, static_cast<size_t>(V) * H * elem, st);
     return e == cudaSuccess ? FLCE_OK : cuda_fail(e);
   }
+  // bf16 outputs: the gradient is computed into fp32 scratch (overwritten, not
+  // accumulated) and rounded once into the caller's buffer afterwards.
+  char* wsb = static_cast<char*>(workspace);
+  float* dh32 = (flags & FLCE_DHIDDEN_BF16) ? reinterpret_cast<float*>(wsb + gs.dh) : d_hidden;
+  float* dw32 = (flags & FLCE_DWEIGHT_BF16) ? reinterpret_cast<float*>(wsb + gs.dw) : d_weight;
+  int32_t inner = flags & (FLCE_ACCUMULATE_DHIDDEN | FLCE_ACCUMULATE_DWEIGHT);
+  if (flags & FLCE_DHIDDEN_BF16) inner &= ~FLCE_ACCUMULATE_DHIDDEN;
+  if (flags & FLCE_DWEIGHT_BF16) inner &= ~FLCE_ACCUMULATE_DWEIGHT;
   if (!(dtype == FLCE_BF16 && bwd_compact())) {  // the compaction checks the labels itself
     e = launch(kHelper, st, [&] {
       label_range_kernel<<<static_cast<unsigned>((N + 255) / 256), 256, 0, st>>>(
@@ -914,11 +951,32 @@ flce_status flce_backward(const void* hidden, const void* weight, const int64_t*
     nv = out;
   }
   if (dtype == FLCE_BF16)
-    return backward_bf16(d, hidden, weight, labels, lse, N, H, V, ignore_index, softcap,
-                         reduction, grad_output, grad_scale, nv, own_count, d_hidden, d_weight,
-                         flags, workspace, st);
-  return backward_fp32(d, hidden, weight, labels, lse, N, H, V, ignore_index, softcap, reduction,
-                       grad_output, grad_scale, nv, d_hidden, d_weight, flags, st);
+    s = backward_bf16(d, hidden, weight, labels, lse, N, H, V, ignore_index, softcap, reduction,
+                      grad_output, grad_scale, nv, own_count, dh32, dw32, inner, workspace, st);
+  else
+    s = backward_fp32(d, hidden, weight, labels, lse, N, H, V, ignore_index, softcap, reduction,
+                      grad_output, grad_scale, nv, dh32, dw32, inner, st);
+  if (s != FLCE_OK) return s;
+  const struct {
+    int32_t flag, acc;
+    const float* src;
+    void* dst;
+    size_t n;
+  } outs[2] = {{FLCE_DHIDDEN_BF16, FLCE_ACCUMULATE_DHIDDEN, dh32, d_hidden,
+                static_cast<size_t>(N) * H},
+               {FLCE_DWEIGHT_BF16, FLCE_ACCUMULATE_DWEIGHT, dw32, d_weight,
+                static_cast<size_t>(V) * H}};
+  for (const auto& o : outs) {
+    if (!(flags & o.flag)) continue;
+    const unsigned blocks = static_cast<unsigned>(
+        std::min<size_t>((o.n / 8 + 255) / 256 + 1, static_cast<size_t>(d->sms) * 8));
+    e = launch(kHelper, st, [&] {
+      f32_to_bf16_kernel<<<blocks, 256, 0, st>>>(o.src, static_cast<__nv_bfloat16*>(o.dst), o.n,
+                                                 (flags & o.acc) ? 1 : 0);
+    });
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return FLCE_OK;
 }
 
 flce_status flce_get_status(const void* workspace, void* stream) {

@@ -160,6 +160,47 @@ __global__ void __launch_bounds__(256)
   if (y != ignore_index && (y < 0 || y >= V)) atomicOr(status, kStatusLabelRange);
 }
 
+// ------------------------------------------------------------------ bf16 outputs
+// dst[i] = bf16(src[i]) or, accumulating, bf16(float(dst[i]) + src[i]); one
+// round-to-nearest-even per element.  8 elements per thread step when both
+// pointers are 16-byte aligned, else one.
+__global__ void __launch_bounds__(256)
+    f32_to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, size_t n,
+                       int accumulate) {
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  const size_t t = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const bool vec = ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15u) == 0;
+  size_t done = 0;
+  if (vec) {
+    const size_t n8 = n / 8;
+    for (size_t i = t; i < n8; i += stride) {
+      const float4 a = reinterpret_cast<const float4*>(src)[2 * i];
+      const float4 b = reinterpret_cast<const float4*>(src)[2 * i + 1];
+      float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      uint4 o;
+      __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(&o);
+      if (accumulate) {
+        const uint4 old = reinterpret_cast<const uint4*>(dst)[i];
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&old);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __bfloat1622float2(p2[k]);
+          v[2 * k] += f.x;
+          v[2 * k + 1] += f.y;
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) o2[k] = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+      reinterpret_cast<uint4*>(dst)[i] = o;
+    }
+    done = n8 * 8;
+  }
+  for (size_t i = done + t; i < n; i += stride) {
+    const float v = src[i] + (accumulate ? __bfloat162float(dst[i]) : 0.0f);
+    dst[i] = __float2bfloat16_rn(v);
+  }
+}
+
 // ------------------------------------------------------------------ row compaction
 // The backward skips token rows whose label is ignore_index (their gradient is
 // exactly zero).  A stable compaction puts the valid rows first, in order, then

@@ -68,14 +68,18 @@ def _prep(hidden: torch.Tensor, weight: torch.Tensor, labels: torch.Tensor):
     return h2, weight.contiguous(), y
 
 
-def workspace_bytes(N: int, H: int, V: int, dtype: torch.dtype = torch.bfloat16) -> int:
-    return int(_lib().flce_workspace_bytes(N, H, V, _DTYPES[dtype]))
+def workspace_bytes(N: int, H: int, V: int, dtype: torch.dtype = torch.bfloat16,
+                    flags: int = 0) -> int:
+    """Workspace for forward/backward; `flags` as for backward (bf16 gradient
+    outputs need fp32 scratch)."""
+    return int(_lib().flce_workspace_bytes_ex(N, H, V, _DTYPES[dtype], int(flags)))
 
 
-def alloc_workspace(N: int, H: int, V: int, dtype: torch.dtype, device) -> torch.Tensor:
-    n = workspace_bytes(N, H, V, dtype)
+def alloc_workspace(N: int, H: int, V: int, dtype: torch.dtype, device,
+                    flags: int = 0) -> torch.Tensor:
+    n = workspace_bytes(N, H, V, dtype, flags)
     if n == 0:
-        raise ValueError("invalid FLCE sizes")
+        raise ValueError("invalid FLCE sizes or flags")
     return torch.empty(n, dtype=torch.uint8, device=device)
 
 
@@ -116,29 +120,38 @@ def backward(hidden: torch.Tensor, weight: torch.Tensor, labels: torch.Tensor,
              workspace: Optional[torch.Tensor] = None,
              d_hidden: Optional[torch.Tensor] = None, d_weight: Optional[torch.Tensor] = None,
              accumulate_d_hidden: bool = False, accumulate_d_weight: bool = False,
+             grad_dtype: torch.dtype = torch.float32,
              check_status: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
-    """dHidden [N, H] and dWeight [V, H] (float32).  With accumulate_* the
-    gradient is added into the given d_hidden / d_weight instead of
-    overwriting them (e.g. over the micro-batches of one optimizer step)."""
+    """dHidden [N, H] and dWeight [V, H], float32 or bfloat16 (the dtype of a
+    given d_hidden / d_weight, else `grad_dtype`).  A bf16 gradient is
+    computed in fp32 and rounded once.  With accumulate_* the gradient is
+    added into the given d_hidden / d_weight instead of overwriting them (e.g.
+    over the micro-batches of one optimizer step)."""
     h2, w, y = _prep(hidden, weight, labels)
     N, H = h2.shape
     V = w.shape[0]
     dev = h2.device
-    if workspace is None:
-        workspace = alloc_workspace(N, H, V, h2.dtype, dev)
+    if grad_dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("grad_dtype must be float32 or bfloat16")
     for name, t, acc, shape in (("d_hidden", d_hidden, accumulate_d_hidden, (N, H)),
                                 ("d_weight", d_weight, accumulate_d_weight, (V, H))):
         if acc and t is None:
             raise ValueError(f"accumulating needs an existing {name}")
-        if t is not None and (tuple(t.shape) != shape or t.dtype != torch.float32
+        if t is not None and (tuple(t.shape) != shape
+                              or t.dtype not in (torch.float32, torch.bfloat16)
                               or not t.is_contiguous() or t.device != dev):
-            raise ValueError(f"{name} must be a contiguous float32 {list(shape)} tensor on {dev}")
+            raise ValueError(f"{name} must be a contiguous float32 or bfloat16 {list(shape)} "
+                             f"tensor on {dev}")
     if d_hidden is None:
-        d_hidden = torch.empty((N, H), dtype=torch.float32, device=dev)
+        d_hidden = torch.empty((N, H), dtype=grad_dtype, device=dev)
     if d_weight is None:
-        d_weight = torch.empty((V, H), dtype=torch.float32, device=dev)
+        d_weight = torch.empty((V, H), dtype=grad_dtype, device=dev)
     flags = ((_native.ACCUMULATE_DHIDDEN if accumulate_d_hidden else 0)
-             | (_native.ACCUMULATE_DWEIGHT if accumulate_d_weight else 0))
+             | (_native.ACCUMULATE_DWEIGHT if accumulate_d_weight else 0)
+             | (_native.DHIDDEN_BF16 if d_hidden.dtype == torch.bfloat16 else 0)
+             | (_native.DWEIGHT_BF16 if d_weight.dtype == torch.bfloat16 else 0))
+    if workspace is None:
+        workspace = alloc_workspace(N, H, V, h2.dtype, dev, flags)
     if grad_output is not None:
         grad_output = grad_output.reshape(()).to(device=dev, dtype=torch.float32).contiguous()
     if num_valid is not None:
@@ -168,10 +181,13 @@ class _FlceFunction(torch.autograd.Function):
     def backward(ctx, grad_loss, _grad_ntok):
         hidden, weight, labels, lse = ctx.saved_tensors
         ignore_index, softcap, reduction, grad_scale, hshape = ctx.cfg
-        dh, dw = backward(hidden, weight, labels, lse, grad_output=grad_loss,
-                          grad_scale=grad_scale, ignore_index=ignore_index, softcap=softcap,
-                          reduction=reduction)
-        return dh.reshape(hshape), dw, None, None, None, None, None
+        # gradients in the parameters' own dtype (bf16 rounded once from fp32)
+        dh = torch.empty(hshape, dtype=hidden.dtype, device=hidden.device).view(-1, hshape[-1])
+        dw = torch.empty(weight.shape, dtype=weight.dtype, device=weight.device)
+        backward(hidden, weight, labels, lse, grad_output=grad_loss, grad_scale=grad_scale,
+                 ignore_index=ignore_index, softcap=softcap, reduction=reduction,
+                 d_hidden=dh, d_weight=dw)
+        return dh.view(hshape), dw, None, None, None, None, None
 
 
 def fused_linear_cross_entropy(hidden, weight, labels, ignore_index: int = -100,

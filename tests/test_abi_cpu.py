@@ -60,6 +60,16 @@ def test_workspace_bytes(lib):
     assert 384 * 2 ** 20 <= big < 386 * 2 ** 20
     assert ws(0, 64, 512, 0) > 0
     assert ws(64, 64, 512, 1) > 0
+    ex = lib.flce_workspace_bytes_ex
+    for dtype in (0, 1):
+        base = ws(300, 64, 1000, dtype)
+        assert ex(300, 64, 1000, dtype, 0) == base
+        assert ex(300, 64, 1000, dtype, 3) == base  # accumulate flags need no scratch
+        assert ex(300, 64, 1000, dtype, 4) >= base + 4 * 300 * 64
+        assert ex(300, 64, 1000, dtype, 8) >= base + 4 * 1000 * 64
+        assert ex(300, 64, 1000, dtype, 12) >= base + 4 * 1300 * 64
+        assert ex(300, 64, 1000, dtype, 16) == 0
+    assert ex(-1, 64, 1000, 0, 4) == 0
 
 
 def _fwd(lib, N=64, H=64, V=512, softcap=0.0, reduction=0, dtype=0, ws_size=None,
@@ -91,8 +101,12 @@ def test_argument_errors_are_synchronous(lib):
                                 float("nan"), None, FAKE, FAKE, 0, FAKE, wsb, None)
     assert bad_bwd == ARG
     bad_flags = lib.flce_backward(FAKE, FAKE, FAKE, FAKE, 64, 64, 512, -100, 0.0, 0, 0, None,
-                                  1.0, None, FAKE, FAKE, 4, FAKE, wsb, None)
+                                  1.0, None, FAKE, FAKE, 16, FAKE, wsb, None)
     assert bad_flags == ARG
+    # bf16 gradient outputs need the larger workspace of flce_workspace_bytes_ex
+    for flags in (4, 8, 12):
+        assert lib.flce_backward(FAKE, FAKE, FAKE, FAKE, 64, 64, 512, -100, 0.0, 0, 0, None,
+                                 1.0, None, FAKE, FAKE, flags, FAKE, wsb, None) == WS
     assert lib.flce_get_status(None, None) == ARG
 
 

@@ -267,3 +267,39 @@ def test_label_term_is_exact(case):
     assert G.rel_l2(got["dh"], rb["d_hidden"]) <= 4e-4
     assert G.rel_l2(got["dw"], rb["d_weight"]) <= 4e-4
     assert np.array_equal(got["dh"], again["dh"]) and np.array_equal(got["dw"], again["dw"])
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_bf16_gradient_outputs(dtype):
+    """bf16 dHidden / dWeight are the fp32 gradients rounded once to nearest even:
+    bf16(g) when overwriting, bf16(float(old) + g) when accumulating."""
+    inp = G.small_inputs(N=700, H=136 if dtype == "bf16" else 64, V=1300, seed=23, n_ign=90,
+                         w_std=0.1)
+    if dtype == "bf16":
+        h, W = G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits)
+    else:
+        h, W = G.f32_tensor(inp.hidden_raw), G.f32_tensor(inp.weight_raw)
+    y = G.labels_tensor(inp.labels)
+    with G.chunks(*SMALL_CHUNKS):
+        f = flce.forward(h, W, y, softcap=2.0, check_status=True)
+        args = dict(softcap=2.0, grad_scale=0.3, check_status=True)
+        dh32, dw32 = flce.backward(h, W, y, f.lse, **args)
+        dh16, dw16 = flce.backward(h, W, y, f.lse, grad_dtype=torch.bfloat16, **args)
+        assert dh16.dtype == torch.bfloat16 and dw16.dtype == torch.bfloat16
+        assert torch.equal(dh16, dh32.to(torch.bfloat16))
+        assert torch.equal(dw16, dw32.to(torch.bfloat16))
+        assert torch.all(dh16[G.labels_tensor(inp.labels) == IGN] == 0)
+        g = torch.Generator(device="cuda").manual_seed(5)
+        old_h = torch.randn(dh32.shape, device="cuda", generator=g).to(torch.bfloat16)
+        old_w = torch.randn(dw32.shape, device="cuda", generator=g).to(torch.bfloat16)
+        acc_h, acc_w = old_h.clone(), old_w.clone()
+        flce.backward(h, W, y, f.lse, d_hidden=acc_h, d_weight=acc_w, accumulate_d_hidden=True,
+                      accumulate_d_weight=True, **args)
+        assert torch.equal(acc_h, (old_h.float() + dh32).to(torch.bfloat16))
+        assert torch.equal(acc_w, (old_w.float() + dw32).to(torch.bfloat16))
+        # mixed: fp32 dHidden accumulated, bf16 dWeight overwritten
+        mix_h, mix_w = dh32.clone(), torch.empty_like(dw16)
+        flce.backward(h, W, y, f.lse, d_hidden=mix_h, d_weight=mix_w, accumulate_d_hidden=True,
+                      **args)
+        assert torch.equal(mix_w, dw16)
+        assert G.rel_l2(mix_h.cpu().numpy(), 2 * dh32.cpu().numpy().astype(np.float64)) <= 1e-6
