@@ -154,3 +154,45 @@ def test_microbatch_token_weighted_scale():
     torch.cuda.synchronize()
     _check_sampled(inp, gold, lse_all.cpu().numpy(), dh_all.cpu().numpy(),
                    dw_acc.cpu().numpy(), gs, seed=5)
+
+
+def test_flat_offsets_beyond_int32():
+    """V*H > 2^31: the top vocabulary rows of W and dWeight lie past the int32
+    range of flat element offsets.  Half of the valid rows take labels there, so
+    the dZ label entries, the dHidden W-row gathers and the dWeight label-term
+    sums all touch those rows; lse and the loss are checked on every row and
+    dWeight on the top rows (plus a sample), against the oracle on vocabulary
+    slices combined by the logsumexp identity lse = log(sum_k exp(lse_k))."""
+    N, H, V = 256, 4096, (1 << 19) + 512  # V*H = 2^31 + 2^21 elements
+    w = fi.custom_workload(N, H, V, seed=41, w_std=0.02, ignore_count=16)
+    inp = fi.make_inputs(w)
+    y = inp.labels.copy()
+    valid = np.nonzero(y != IGN)[0]
+    rng = np.random.default_rng(7)
+    y[valid[::2]] = rng.integers(V - 512, V, size=len(valid[::2]))
+    h = G.bf16_tensor(inp.hidden_bits)
+    W = G.bf16_tensor(inp.weight_bits)
+    yt = G.labels_tensor(y)
+    f = flce.forward(h, W, yt, IGN, 0.0, "sum", check_status=True)
+    dh, dw = flce.backward(h, W, yt, f.lse, check_status=True)
+    torch.cuda.synchronize()
+    lse_gpu = f.lse.cpu().numpy()
+    top = torch.arange(V - 512, V, device="cuda")
+    low = torch.from_numpy(np.sort(rng.choice(V - 512, size=64, replace=False))).cuda()
+    vrows = torch.cat([low, top])
+    dw_rows = dw[vrows].cpu().numpy()
+    dh_np = dh.cpu().numpy()
+    loss = f.loss.item()
+    del dw, dh, W
+    torch.cuda.empty_cache()
+    parts = [oracle.lse_rows(inp.hidden, inp.weight[a:a + 65536], np.arange(N))
+             for a in range(0, V, 65536)]
+    lse_ref = np.logaddexp.reduce(np.stack(parts), axis=0)
+    assert np.max(np.abs(lse_gpu - lse_ref)) <= G.LSE_ATOL
+    ll = oracle.label_logits(inp.hidden, inp.weight, y, IGN)
+    G.check_loss(loss, float(np.sum((lse_ref - ll)[y != IGN])))
+    ref_dw = oracle.d_weight_rows(inp.hidden, inp.weight, y, vrows.cpu().numpy(), lse_ref, 1.0,
+                                  IGN)
+    assert G.rel_l2(dw_rows, ref_dw) <= G.GRAD_RL2
+    assert G.rel_l2(dw_rows[64:], ref_dw[64:]) <= G.GRAD_RL2  # the rows past 2^31
+    assert np.all(dh_np[y == IGN] == 0.0) and np.all(np.isfinite(dh_np))
