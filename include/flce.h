@@ -134,8 +134,8 @@ flce_status flce_forward(const void* hidden, const void* weight, const int64_t* 
  * (each with grad_scale = 1 / the step's total non-ignored count) gives the
  * token-weighted gradient of the whole batch (modelscope/twinkle PR #335,
  * item 2).  The call clears the workspace status word and records in it a
- * label outside [0, V) that is not ignore_index (FLCE_ERR_LABEL_RANGE; such a
- * row contributes only its softmax term, as in the forward). */
+ * label outside [0, V) that is not ignore_index (FLCE_ERR_LABEL_RANGE); such a
+ * row is treated as ignored (zero gradient, not counted), as in the forward. */
 flce_status flce_backward(const void* hidden, const void* weight, const int64_t* labels,
                           const float* lse, int64_t N, int64_t H, int64_t V,
                           int64_t ignore_index, float softcap, int32_t reduction, int32_t dtype,

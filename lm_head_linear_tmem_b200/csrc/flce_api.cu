@@ -725,11 +725,11 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
       if (softcap > 0.f) {
         DzEpi<true>::Params ep{lab,  lsev,    ignore_index, static_cast<int>(t0),
                                rows, static_cast<int>(v0), cols, softcap, 1.0f / softcap,
-                               resid};
+                               resid, V};
         e = run_gemm<DzEpi<true>, false, false>(d, kSlotDzCap, kBwdDz, pz, ep, nullptr, ep, st);
       } else {
         DzEpi<false>::Params ep{lab,  lsev, ignore_index, static_cast<int>(t0), rows,
-                                static_cast<int>(v0), cols, 0.f, 0.f, resid};
+                                static_cast<int>(v0), cols, 0.f, 0.f, resid, V};
         e = run_gemm<DzEpi<false>, false, false>(d, kSlotDz, kBwdDz, pz, ep, nullptr, ep, st);
       }
       if (e != cudaSuccess) return cuda_fail(e);
@@ -945,7 +945,7 @@ flce_status flce_backward(const void* hidden, const void* weight, const int64_t*
     long long* out = ws_nvalid(workspace);
     e = launch(kHelper, st, [&] {
       count_valid_kernel<<<1, kFinalThreads, 0, st>>>(labels, static_cast<int>(N), ignore_index,
-                                                      out);
+                                                      V, out);
     });
     if (e != cudaSuccess) return cuda_fail(e);
     nv = out;

@@ -132,14 +132,17 @@ __global__ void __launch_bounds__(kFinalThreads)
   }
 }
 
-// n = #rows with label != ignore_index (one block).
+// n = #rows whose label is neither ignore_index nor outside [0, V) (one block).
 __global__ void __launch_bounds__(kFinalThreads)
     count_valid_kernel(const int64_t* __restrict__ labels, int N, int64_t ignore_index,
-                       long long* n_valid_out) {
+                       int64_t V, long long* n_valid_out) {
   __shared__ long long sc[kFinalThreads];
   const int t = threadIdx.x;
   long long c = 0;
-  for (int i = t; i < N; i += kFinalThreads) c += (labels[i] != ignore_index) ? 1 : 0;
+  for (int i = t; i < N; i += kFinalThreads) {
+    const int64_t y = labels[i];
+    c += (y != ignore_index && y >= 0 && y < V) ? 1 : 0;
+  }
   sc[t] = c;
   __syncthreads();
   for (int w = kFinalThreads / 2; w > 0; w >>= 1) {
@@ -203,7 +206,8 @@ __global__ void __launch_bounds__(256)
 
 // ------------------------------------------------------------------ row compaction
 // The backward skips token rows whose label is ignore_index (their gradient is
-// exactly zero).  A stable compaction puts the valid rows first, in order, then
+// exactly zero), and rows whose label lies outside [0, V) (an error the status
+// word reports; the forward leaves them out of the loss and the count too).  A stable compaction puts the valid rows first, in order, then
 // the ignored rows, in order: perm[j] is the original row of compact row j.
 constexpr int kCompactThreads = 1024;
 
@@ -215,8 +219,9 @@ __global__ void __launch_bounds__(kCompactThreads)
   __shared__ int warp_sum[kCompactThreads / 32];
   const int i = blockIdx.x * kCompactThreads + threadIdx.x;
   const int64_t y = (i < N) ? labels[i] : ignore_index;
-  const bool v = (i < N) && (y != ignore_index);
-  if (v && (y < 0 || y >= V)) atomicOr(status, kStatusLabelRange);
+  const bool in_range = y >= 0 && y < V;
+  if (i < N && y != ignore_index && !in_range) atomicOr(status, kStatusLabelRange);
+  const bool v = (i < N) && (y != ignore_index) && in_range;  // out of range: as ignored
   const unsigned m = __ballot_sync(0xffffffffu, v);
   if ((threadIdx.x & 31) == 0) warp_sum[threadIdx.x >> 5] = __popc(m);
   __syncthreads();
@@ -270,7 +275,7 @@ __global__ void __launch_bounds__(kCompactThreads)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int i = blockIdx.x * kCompactThreads + threadIdx.x;
   const int64_t y = (i < N) ? labels[i] : ignore_index;
-  const bool v = (i < N) && (y != ignore_index);
+  const bool v = (i < N) && (y != ignore_index) && y >= 0 && y < V;
   const unsigned m = __ballot_sync(0xffffffffu, v);
   if (lane == 0) warp_sum[warp] = __popc(m);
   __syncthreads();
@@ -282,8 +287,8 @@ __global__ void __launch_bounds__(kCompactThreads)
     perm[j] = i;
     labels_c[j] = v ? y : ignore_index;
     lse_c[j] = v ? lse[i] : 0.f;
-    if (v) {  // labels outside [0, V) share the key V and are sorted last
-      sort_keys[j] = static_cast<uint32_t>((y >= 0 && y < V) ? y : V);
+    if (v) {  // the key is the label (in [0, V) for every compacted row)
+      sort_keys[j] = static_cast<uint32_t>(y);
       sort_vals[j] = i;
     }
   }
@@ -614,7 +619,7 @@ __global__ void __launch_bounds__(kSimtThreads)
   const int row = blockIdx.x;
   const int t = threadIdx.x;
   const int64_t y = labels[row];
-  const bool valid = (y != ignore_index);
+  const bool valid = (y != ignore_index) && y >= 0 && y < V;  // out of range: as ignored
   const float g = simt_grad_scale(grad_output, grad_scale, n_valid, mean);
   const float l = lse[row];
   for (int k = t; k < H; k += kSimtThreads) {
@@ -681,7 +686,7 @@ __global__ void __launch_bounds__(kSimtThreads)
       const int i = i0 + t;
       const int64_t y = labels[i];
       float gz = 0.f;
-      if (y != ignore_index) {
+      if (y != ignore_index && y >= 0 && y < V) {  // out of range: as ignored
         const float* hi = hidden + static_cast<size_t>(i) * H;
         float z = 0.f;
         for (int k = 0; k < H; ++k) z = fmaf(hi[k], w[k], z);

@@ -229,7 +229,8 @@ struct DzEpi {
     int cols;   // valid vocab columns in this block
     float softcap;
     float inv_softcap;
-    float* resid;  // [token rows] or null
+    float* resid;      // [token rows] or null
+    int64_t v_total;   // V: a label outside [0, V) counts as ignored
   };
 
   __device__ static void tile(const Params& p, const GemmArgs&, int m_base, int nb,
@@ -250,7 +251,7 @@ struct DzEpi {
     if (row_l < p.rows) {
       const int row = p.t0 + row_l;
       const int64_t y = p.labels[row];
-      valid = (y != p.ignore_index);
+      valid = (y != p.ignore_index) && y >= 0 && y < p.v_total;
       const int64_t c0 = static_cast<int64_t>(p.v0) + static_cast<int64_t>(nb) * BN;
       if (valid && y >= c0 && y < c0 + BN) y_local = static_cast<int>(y - c0);
       lse2 = p.lse[row] * kLog2e;

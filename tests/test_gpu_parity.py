@@ -135,20 +135,29 @@ def test_label_out_of_range_is_reported():
                      G.labels_tensor(y), check_status=True)
     assert e.value.status == 3
     # the backward finds the same label on its own (compacted bf16, uncompacted, fp32)
+    # and, like the forward, treats its row as ignored: the gradients equal, bit for
+    # bit, those of the labels with that row set to ignore_index
+    y_ign = y.copy()
+    y_ign[5] = IGN
+    for dt in ("bf16", "fp32"):
+        if dt == "bf16":
+            h, W = G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits)
+        else:
+            h, W = G.f32_tensor(inp.hidden_raw), G.f32_tensor(inp.weight_raw)
+        lse = flce.forward(h, W, G.labels_tensor(y_ign), reduction="mean", check_status=True).lse
+        for env in (("1", "0") if dt == "bf16" else ("1",)):
+            os.environ["FLCE_BWD_COMPACT"] = env
+            try:
+                ref = flce.backward(h, W, G.labels_tensor(y_ign), lse, reduction="mean",
+                                    check_status=True)
+                ws = flce.alloc_workspace(130, 64, 300, h.dtype, "cuda")
+                got = flce.backward(h, W, G.labels_tensor(y), lse, reduction="mean",
+                                    workspace=ws)
+                assert flce.status(ws) == 3
+                assert torch.equal(got[0], ref[0]) and torch.equal(got[1], ref[1])
+            finally:
+                os.environ.pop("FLCE_BWD_COMPACT", None)
     h, W = G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits)
-    lse = torch.zeros(130, device="cuda")
-    for env in ("1", "0"):
-        os.environ["FLCE_BWD_COMPACT"] = env
-        try:
-            with pytest.raises(flce.FlceError) as e:
-                flce.backward(h, W, G.labels_tensor(y), lse, check_status=True)
-            assert e.value.status == 3
-        finally:
-            os.environ.pop("FLCE_BWD_COMPACT", None)
-    with pytest.raises(flce.FlceError) as e:
-        flce.backward(G.f32_tensor(inp.hidden_raw), G.f32_tensor(inp.weight_raw),
-                      G.labels_tensor(y), lse, check_status=True)
-    assert e.value.status == 3
     # the status is cleared by the next forward ...
     f = flce.forward(h, W, G.labels_tensor(inp.labels), check_status=True)
     # ... and by the next backward, also on a workspace never used before
