@@ -619,10 +619,10 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
             labels, lse, n, ignore_index, block_valid, n_valid_c, perm, labels_c, lse_c, V,
             keys[0], vals[0]);
       });
-    // Valid rows in (label, token) order: keys are labels, or V for a label
-    // outside [0, V), so ceil(bits(V) / 8) passes of 8 bits sort them.
+    // Valid rows in (label, token) order: keys are labels in [0, V), so
+    // ceil(bits(V - 1) / 8) passes of 8 bits sort them.
     int key_bits = 0;
-    while ((V >> key_bits) != 0) ++key_bits;
+    while (((V - 1) >> key_bits) != 0) ++key_bits;
     const int passes = (key_bits + 7) / 8;
     int* hist = reinterpret_cast<int*>(w + BL.hist);
     for (int ps = 0; ps < passes && e == cudaSuccess; ++ps) {

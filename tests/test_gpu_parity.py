@@ -337,3 +337,28 @@ def test_large_logits_stay_finite(softcap):
     assert np.all(got["dh"][inp.labels == IGN] == 0.0)
     assert G.rel_l2(got["dh"], rb["d_hidden"]) <= G.GRAD_RL2
     assert G.rel_l2(got["dw"], rb["d_weight"]) <= G.GRAD_RL2
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("N,H,V", [(37, 8, 2), (37, 8, 7), (300, 16, 1), (129, 24, 257)])
+def test_degenerate_shapes(N, H, V, dtype):
+    """The smallest hidden size (H = 8), one- and two-word vocabularies, and a
+    vocabulary one past a tile: the tensor maps' boxes extend far past the tensors."""
+    inp = G.small_inputs(N=N, H=H, V=V, seed=25 + V, n_ign=N // 5, w_std=0.5)
+    if dtype == "bf16":
+        h, W = G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits)
+        hid, wt = inp.hidden, inp.weight
+    else:
+        h, W = G.f32_tensor(inp.hidden_raw), G.f32_tensor(inp.weight_raw)
+        hid, wt = inp.hidden_raw, inp.weight_raw
+    got = run(h, W, G.labels_tensor(inp.labels), 0.0, "sum")
+    if V == 1:
+        # every valid row's loss is lse - L_y = 0 and its gradient 0 - 0; fp32 keeps
+        # only rounding-level residue of the log2-domain logsumexp
+        rf = oracle.forward(hid, wt, inp.labels, IGN, 0.0, "sum")
+        assert got["ntok"] == rf["num_tokens"]
+        assert abs(got["loss"]) <= 1e-5 * np.sum(np.abs(rf["lse"]))
+        assert np.max(np.abs(got["lse"] - rf["lse"])) <= G.LSE_ATOL
+        assert np.max(np.abs(got["dh"])) <= 1e-5 and np.max(np.abs(got["dw"])) <= 1e-5
+    else:
+        compare(got, hid, wt, inp.labels, 0.0, "sum")
