@@ -50,7 +50,11 @@
  *    dtype FLCE_FP32: hidden/weight hold float32; a CUDA-core path runs
  *    (a correctness path for small problems, not tuned).
  *  - stream is a cudaStream_t (NULL = legacy default stream).  Every call is
- *    asynchronous on that stream and returns after enqueueing its kernels.
+ *    asynchronous on that stream and returns after enqueueing its kernels,
+ *    without synchronising, so flce_forward and flce_backward may be captured
+ *    into a CUDA graph (after one uncaptured call with the same shapes, which
+ *    sets the kernels' shared-memory attributes) and replayed with the inputs
+ *    updated in place; flce_get_status synchronises and must stay outside.
  *  - The caller owns every buffer, including the workspace (at least
  *    flce_workspace_bytes(...) bytes, 256-byte aligned).  The library does not
  *    allocate device memory and keeps no per-call state.  Calls that share a
