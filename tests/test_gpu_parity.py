@@ -362,3 +362,21 @@ def test_degenerate_shapes(N, H, V, dtype):
         assert np.max(np.abs(got["dh"])) <= 1e-5 and np.max(np.abs(got["dw"])) <= 1e-5
     else:
         compare(got, hid, wt, inp.labels, 0.0, "sum")
+
+
+@pytest.mark.parametrize("switch", ["FLCE_CTA_GROUP=1", "FLCE_BWD_FUSE=0", "FLCE_BWD_COMPACT=0",
+                                    "FLCE_MN3D=0"])
+def test_alternative_paths(switch):
+    """Each A/B switch of the library selects another correct path: single-CTA
+    128 x 256 tiles, separate dHidden and dWeight launches, no row compaction (and
+    so no exact label term), 2-D views for MN-major operands."""
+    key, val = switch.split("=")
+    inp = G.small_inputs(N=2100, H=192, V=4500, seed=26, n_ign=300, w_std=0.1)
+    os.environ[key] = val
+    try:
+        with G.chunks(*SMALL_CHUNKS):
+            got = run(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
+                      G.labels_tensor(inp.labels), 2.0, "mean", grad_scale=0.7)
+    finally:
+        os.environ.pop(key, None)
+    compare(got, inp.hidden, inp.weight, inp.labels, 2.0, "mean", grad_scale=0.7)
