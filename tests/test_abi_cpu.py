@@ -3,6 +3,7 @@ declares; host-side argument checks answer without touching a GPU."""
 import ctypes
 import os
 import re
+import subprocess
 
 import pytest
 
@@ -117,3 +118,12 @@ def test_profile_api_host_side(lib):
     assert n.value == 0
     assert lib.flce_profile_read(99, ctypes.byref(ms), ctypes.byref(n)) == 1
     assert lib.flce_profile_enable(0) == 0
+
+
+def test_header_is_plain_c_and_a_c_program_links(tmp_path):
+    """include/flce.h compiles as C99 with all warnings as errors, and a C caller
+    links against the library and the CUDA runtime (it runs in the GPU tests)."""
+    from tests import _c_driver
+    exe = _c_driver.build_driver(str(tmp_path))
+    res = subprocess.run([exe], capture_output=True, text=True)
+    assert res.returncode == 1 and "usage" in res.stderr  # no GPU call without arguments
