@@ -390,6 +390,17 @@ def run_own(args, rank, world, local_rank):
                     "peak_source": f"{peak_src} bf16_tflops_sustained",
                     "traffic": dram_traffic(dom),
                     "per_launch_flops": per_launch_flops, "avg_launch_ms": avg_ms}
+    # every tensor-core kernel kind against the same peak (the dominant one is `roofline`)
+    gemm_roofline = {}
+    for kind, fl in credited.items():
+        if kind in kinds:
+            avg = kinds[kind]["ms_total"] / kinds[kind]["launches"]
+            ach = fl * args.steps / kinds[kind]["launches"] / (avg / 1e3) / 1e12
+            gemm_roofline[kind] = {"achieved_tflops": ach, "avg_launch_ms": avg,
+                                   "frac_of_sustained": ach / float(peaks.get(
+                                       "bf16_tflops_sustained",
+                                       FALLBACK_PEAKS["bf16_tflops_sustained"])),
+                                   "dram_bytes_per_launch": dram_traffic(kind)}
     tflops = flops_step / (ms_step / 1e3) / 1e12
     burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     sust = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
@@ -416,6 +427,7 @@ def run_own(args, rank, world, local_rank):
                             "backward_rows": n_bwd, "tokens": N,
                             "peak_source": peak_src},
         "roofline": roofline,
+        "gemm_roofline": gemm_roofline,
         "kernels": kinds,
         "kernels_region_ms_per_step": ms_prof / args.steps,
         "cpu_baseline": cpu,
