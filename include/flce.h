@@ -18,7 +18,8 @@
  *                                                  (F.cross_entropy semantics:
  *                                                   modelscope/twinkle PR #335,
  *                                                   "Experiment results")
- *   n     = #rows with y_i != ignore_index
+ *   n     = #rows with y_i != ignore_index (a label outside [0, V) is an error,
+ *           reported asynchronously; its row is treated as ignored)
  *   'sum'  -> loss = sum_i loss_i,             num_tokens = n
  *   'mean' -> loss = sum_i loss_i / max(n, 1), num_tokens = 0
  *                                                  (modelscope/twinkle PR #335,
@@ -34,8 +35,8 @@
  *   g     = grad_output * grad_scale * ('mean' ? 1 / max(n, 1) : 1)
  *   dZ_iv = g * (exp(L_iv - lse_i) - [v == y_i]) * (softcap > 0 ? 1 - (L_iv/softcap)^2 : 1),
  *           0 on ignored rows
- *   d_hidden = dZ . weight        [N, H] float32, overwritten
- *   d_weight = dZ^T . hidden      [V, H] float32, overwritten
+ *   d_hidden = dZ . weight        [N, H] float32 or bf16, overwritten or accumulated
+ *   d_weight = dZ^T . hidden      [V, H] float32 or bf16, overwritten or accumulated
  * grad_scale is the caller's micro-batch / token-count weighting
  * (modelscope/twinkle PR #335, item 2: 1.0 for 'sum' per micro-batch; the
  * trainer divides a 'sum' loss's gradient by the global non-padding token
@@ -180,8 +181,9 @@ flce_status flce_forward_noalloc(const void* hidden, const void* weight, const i
                                  float softcap, int32_t reduction, int32_t dtype, float* loss,
                                  int64_t* num_tokens, float* lse, uint32_t* status, void* stream);
 
-/* Synchronise `stream`, then return the first asynchronous error recorded in
- * the workspace since the last flce_forward (FLCE_OK if none). */
+/* Synchronise `stream`, then return the asynchronous error recorded in the
+ * workspace by the latest flce_forward or flce_backward on it (FLCE_OK if
+ * none; a label-range error is reported before a timeout). */
 flce_status flce_get_status(const void* workspace, void* stream);
 
 /* Self-test of failure reporting: launches one tiny kernel whose thread waits
