@@ -380,3 +380,14 @@ def test_alternative_paths(switch):
     finally:
         os.environ.pop(key, None)
     compare(got, inp.hidden, inp.weight, inp.labels, 2.0, "mean", grad_scale=0.7)
+
+
+@pytest.mark.parametrize("softcap", [0.05, 1.0])
+def test_small_softcap_saturates(softcap):
+    """A softcap well below the logits' spread saturates tanh: most capped logits sit at
+    +-softcap and their derivative 1 - tanh^2 vanishes; the rest still carry the
+    gradient."""
+    inp = G.small_inputs(N=300, H=200, V=1000, seed=28, n_ign=30, w_std=0.2)
+    got = run(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
+              G.labels_tensor(inp.labels), softcap, "mean")
+    compare(got, inp.hidden, inp.weight, inp.labels, softcap, "mean")
