@@ -113,6 +113,18 @@ flce_status flce_forward(const void* hidden, const void* weight, const int64_t* 
                          int32_t reduction, int32_t dtype, float* loss, int64_t* num_tokens,
                          float* lse, void* workspace, size_t workspace_bytes, void* stream);
 
+/* flce_forward with the returned loss multiplied by loss_scale (applied in
+ * float64 before the single rounding to float32; num_tokens and lse are
+ * unchanged).  loss_scale = 1 / n_global normalises a 'sum' loss by a global
+ * non-padding token count (NeMo AutoModel linear_ce API, forward(
+ * num_label_tokens)); the matching backward takes grad_scale = loss_scale.
+ * A NaN or infinite loss_scale is FLCE_ERR_ARG. */
+flce_status flce_forward_ex(const void* hidden, const void* weight, const int64_t* labels,
+                            int64_t N, int64_t H, int64_t V, int64_t ignore_index, float softcap,
+                            int32_t reduction, int32_t dtype, float loss_scale, float* loss,
+                            int64_t* num_tokens, float* lse, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
 /* flce_backward flags. */
 #define FLCE_ACCUMULATE_DHIDDEN 1 /* d_hidden += gradient (else overwritten) */
 #define FLCE_ACCUMULATE_DWEIGHT 2 /* d_weight += gradient (else overwritten) */

@@ -34,6 +34,8 @@ SIGNATURES = {
     "flce_workspace_bytes_ex": (c_size, [c_i64, c_i64, c_i64, c_i32, c_i32]),
     "flce_forward": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32, c_i32,
                              c_i32, c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),
+    "flce_forward_ex": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32, c_i32,
+                                c_i32, c_f32, c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),
     "flce_backward": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32,
                               c_i32, c_i32, c_vp, c_f32, c_vp, c_vp, c_vp, c_i32, c_vp, c_size,
                               c_vp]),

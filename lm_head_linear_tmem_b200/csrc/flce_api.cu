@@ -464,8 +464,9 @@ uint32_t b_box_rows() { return static_cast<uint32_t>(BN / cta_group()); }
 // ---------------------------------------------------------------- forward
 flce_status forward_bf16(DevInfo* d, const void* hidden, const void* weight,
                          const int64_t* labels, int64_t N, int64_t H, int64_t V,
-                         int64_t ignore_index, float softcap, int32_t reduction, float* loss,
-                         int64_t* num_tokens, float* lse, void* ws, cudaStream_t st) {
+                         int64_t ignore_index, float softcap, int32_t reduction,
+                         double loss_scale, float* loss, int64_t* num_tokens, float* lse,
+                         void* ws, cudaStream_t st) {
   char* w = static_cast<char*>(ws);
   const FwdLayout L = fwd_layout(N, V, true);
   float* part_m = reinterpret_cast<float*>(w + L.part_m);
@@ -518,8 +519,8 @@ flce_status forward_bf16(DevInfo* d, const void* hidden, const void* weight,
   if (e != cudaSuccess) return cuda_fail(e);
   e = launch(kFwdMerge, st, [&] {
     finalize_kernel<<<1, kFinalThreads, 0, st>>>(block_loss, block_cnt, nblk,
-                                                 reduction == FLCE_MEAN, loss, num_tokens,
-                                                 ws_nvalid(ws));
+                                                 reduction == FLCE_MEAN, loss_scale, loss,
+                                                 num_tokens, ws_nvalid(ws));
   });
   if (e != cudaSuccess) return cuda_fail(e);
   return FLCE_OK;
@@ -527,8 +528,9 @@ flce_status forward_bf16(DevInfo* d, const void* hidden, const void* weight,
 
 flce_status forward_fp32(DevInfo* d, const void* hidden, const void* weight,
                          const int64_t* labels, int64_t N, int64_t H, int64_t V,
-                         int64_t ignore_index, float softcap, int32_t reduction, float* loss,
-                         int64_t* num_tokens, float* lse, void* ws, cudaStream_t st) {
+                         int64_t ignore_index, float softcap, int32_t reduction,
+                         double loss_scale, float* loss, int64_t* num_tokens, float* lse,
+                         void* ws, cudaStream_t st) {
   (void)d;
   char* w = static_cast<char*>(ws);
   const FwdLayout L = fwd_layout(N, V, false);
@@ -556,8 +558,8 @@ flce_status forward_fp32(DevInfo* d, const void* hidden, const void* weight,
   if (e != cudaSuccess) return cuda_fail(e);
   e = launch(kFwdMerge, st, [&] {
     finalize_kernel<<<1, kFinalThreads, 0, st>>>(block_loss, block_cnt, nblk,
-                                                 reduction == FLCE_MEAN, loss, num_tokens,
-                                                 ws_nvalid(ws));
+                                                 reduction == FLCE_MEAN, loss_scale, loss,
+                                                 num_tokens, ws_nvalid(ws));
   });
   if (e != cudaSuccess) return cuda_fail(e);
   return FLCE_OK;
@@ -871,6 +873,17 @@ flce_status flce_forward(const void* hidden, const void* weight, const int64_t* 
                          int64_t N, int64_t H, int64_t V, int64_t ignore_index, float softcap,
                          int32_t reduction, int32_t dtype, float* loss, int64_t* num_tokens,
                          float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  return flce_forward_ex(hidden, weight, labels, N, H, V, ignore_index, softcap, reduction, dtype,
+                         1.0f, loss, num_tokens, lse, workspace, workspace_bytes, stream);
+}
+
+flce_status flce_forward_ex(const void* hidden, const void* weight, const int64_t* labels,
+                            int64_t N, int64_t H, int64_t V, int64_t ignore_index, float softcap,
+                            int32_t reduction, int32_t dtype, float loss_scale, float* loss,
+                            int64_t* num_tokens, float* lse, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  if (!(loss_scale == loss_scale) || loss_scale == INFINITY || loss_scale == -INFINITY)
+    return FLCE_ERR_ARG;
   flce_status s = check_common(hidden, weight, labels, N, H, V, softcap, reduction, dtype,
                                workspace, workspace_bytes);
   if (s != FLCE_OK) return s;
@@ -890,9 +903,9 @@ flce_status flce_forward(const void* hidden, const void* weight, const int64_t* 
   }
   if (dtype == FLCE_BF16)
     return forward_bf16(d, hidden, weight, labels, N, H, V, ignore_index, softcap, reduction,
-                        loss, num_tokens, lse, workspace, st);
-  return forward_fp32(d, hidden, weight, labels, N, H, V, ignore_index, softcap, reduction, loss,
-                      num_tokens, lse, workspace, st);
+                        loss_scale, loss, num_tokens, lse, workspace, st);
+  return forward_fp32(d, hidden, weight, labels, N, H, V, ignore_index, softcap, reduction,
+                      loss_scale, loss, num_tokens, lse, workspace, st);
 }
 
 flce_status flce_backward(const void* hidden, const void* weight, const int64_t* labels,
@@ -1131,9 +1144,9 @@ extern "C" flce_status flce_forward_noalloc(const void* hidden, const void* weig
   } else {
     s = (dtype == FLCE_BF16)
             ? forward_bf16(d, hidden, weight, labels, N, H, V, ignore_index, softcap, reduction,
-                           loss, num_tokens, lse, ws, st)
+                           1.0, loss, num_tokens, lse, ws, st)
             : forward_fp32(d, hidden, weight, labels, N, H, V, ignore_index, softcap, reduction,
-                           loss, num_tokens, lse, ws, st);
+                           1.0, loss, num_tokens, lse, ws, st);
     if (s != FLCE_OK) return s;
   }
   if (status != nullptr) {

@@ -92,7 +92,8 @@ def status(workspace: torch.Tensor) -> int:
 def forward(hidden: torch.Tensor, weight: torch.Tensor, labels: torch.Tensor,
             ignore_index: int = -100, softcap: float = 0.0, reduction: str = "sum",
             workspace: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-            check_status: bool = False) -> FlceForward:
+            check_status: bool = False, loss_scale: float = 1.0) -> FlceForward:
+    """loss ('sum' or 'mean', times loss_scale), num_tokens and every row's lse."""
     h2, w, y = _prep(hidden, weight, labels)
     N, H = h2.shape
     V = w.shape[0]
@@ -103,10 +104,10 @@ def forward(hidden: torch.Tensor, weight: torch.Tensor, labels: torch.Tensor,
     ntok = torch.empty((), dtype=torch.int64, device=dev)
     if lse is None:
         lse = torch.empty(N, dtype=torch.float32, device=dev)
-    st = _lib().flce_forward(_ptr(h2), _ptr(w), _ptr(y), N, H, V, int(ignore_index),
-                             float(softcap), _REDUCTIONS[reduction], _DTYPES[h2.dtype],
-                             _ptr(loss), _ptr(ntok), _ptr(lse), _ptr(workspace),
-                             workspace.numel(), _stream(dev))
+    st = _lib().flce_forward_ex(_ptr(h2), _ptr(w), _ptr(y), N, H, V, int(ignore_index),
+                                float(softcap), _REDUCTIONS[reduction], _DTYPES[h2.dtype],
+                                float(loss_scale), _ptr(loss), _ptr(ntok), _ptr(lse),
+                                _ptr(workspace), workspace.numel(), _stream(dev))
     _native.check(st, "flce_forward")
     if check_status:
         _native.check(status(workspace), "flce_forward (device status)")
@@ -170,10 +171,13 @@ def backward(hidden: torch.Tensor, weight: torch.Tensor, labels: torch.Tensor,
 
 class _FlceFunction(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, hidden, weight, labels, ignore_index, softcap, reduction, grad_scale):
-        out = forward(hidden, weight, labels, ignore_index, softcap, reduction)
+    def forward(ctx, hidden, weight, labels, ignore_index, softcap, reduction, grad_scale,
+                loss_scale):
+        out = forward(hidden, weight, labels, ignore_index, softcap, reduction,
+                      loss_scale=loss_scale)
         ctx.save_for_backward(hidden, weight, labels, out.lse)
-        ctx.cfg = (ignore_index, softcap, reduction, grad_scale, hidden.shape)
+        # the returned loss is scaled by loss_scale, so is its gradient
+        ctx.cfg = (ignore_index, softcap, reduction, grad_scale * loss_scale, hidden.shape)
         ctx.mark_non_differentiable(out.num_tokens)
         return out.loss, out.num_tokens
 
@@ -187,15 +191,17 @@ class _FlceFunction(torch.autograd.Function):
         backward(hidden, weight, labels, lse, grad_output=grad_loss, grad_scale=grad_scale,
                  ignore_index=ignore_index, softcap=softcap, reduction=reduction,
                  d_hidden=dh, d_weight=dw)
-        return dh.view(hshape), dw, None, None, None, None, None
+        return dh.view(hshape), dw, None, None, None, None, None, None
 
 
 def fused_linear_cross_entropy(hidden, weight, labels, ignore_index: int = -100,
                                softcap: float = 0.0, reduction: str = "sum",
-                               grad_scale: float = 1.0):
-    """Differentiable (loss, num_tokens); gradients flow to hidden and weight."""
+                               grad_scale: float = 1.0, loss_scale: float = 1.0):
+    """Differentiable (loss, num_tokens); gradients flow to hidden and weight.
+    The loss is multiplied by loss_scale (and so is its gradient); grad_scale
+    scales the gradient alone (a micro-batch's token weighting)."""
     return _FlceFunction.apply(hidden, weight, labels, ignore_index, softcap, reduction,
-                               grad_scale)
+                               grad_scale, loss_scale)
 
 
 class FusedLinearCrossEntropy(torch.nn.Module):
@@ -214,9 +220,23 @@ class FusedLinearCrossEntropy(torch.nn.Module):
         self.num_tokens: Optional[torch.Tensor] = None
 
     def forward(self, hidden_states: torch.Tensor, labels: torch.Tensor,
-                lm_weight: torch.Tensor, grad_scale: float = 1.0) -> torch.Tensor:
+                lm_weight: torch.Tensor, num_label_tokens: Optional[int] = None,
+                grad_reduce_group=None, *, grad_scale: float = 1.0) -> torch.Tensor:
+        """Loss of hidden_states [..., H] against labels [...] with lm_weight [V, H].
+
+        num_label_tokens: the global number of non-padding target tokens; a 'sum'
+        loss is divided by max(num_label_tokens, 1) (in the library's fp64 loss
+        sum) and so is its gradient.  Ignored for 'mean'.
+        grad_reduce_group: only None (one GPU, a regular lm_weight tensor).
+        grad_scale: scales the gradient alone (micro-batch token weighting)."""
+        if grad_reduce_group is not None:
+            raise NotImplementedError("a sharded lm_weight (grad_reduce_group) is not "
+                                      "supported: this loss runs on one GPU")
+        loss_scale = 1.0
+        if num_label_tokens is not None and self.reduction == "sum":
+            loss_scale = 1.0 / max(int(num_label_tokens), 1)
         loss, ntok = fused_linear_cross_entropy(hidden_states, lm_weight, labels,
                                                 self.ignore_index, self.logit_softcapping,
-                                                self.reduction, grad_scale)
+                                                self.reduction, grad_scale, loss_scale)
         self.num_tokens = ntok
         return loss

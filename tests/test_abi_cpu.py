@@ -109,6 +109,9 @@ def test_argument_errors_are_synchronous(lib):
         assert lib.flce_backward(FAKE, FAKE, FAKE, FAKE, 64, 64, 512, -100, 0.0, 0, 0, None,
                                  1.0, None, FAKE, FAKE, flags, FAKE, wsb, None) == WS
     assert lib.flce_get_status(None, None) == ARG
+    for bad_scale in (float("nan"), float("inf")):
+        assert lib.flce_forward_ex(FAKE, FAKE, FAKE, 64, 64, 512, -100, 0.0, 0, 0, bad_scale,
+                                   FAKE, FAKE, FAKE, FAKE, wsb, None) == ARG
 
 
 def test_profile_api_host_side(lib):

@@ -391,3 +391,31 @@ def test_small_softcap_saturates(softcap):
     got = run(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
               G.labels_tensor(inp.labels), softcap, "mean")
     compare(got, inp.hidden, inp.weight, inp.labels, softcap, "mean")
+
+
+def test_module_num_label_tokens():
+    """NeMo AutoModel linear_ce API, forward(num_label_tokens): the global count of
+    non-padding target tokens normalises a 'sum' loss (and so its gradient); it is
+    not used by 'mean'; a sharded lm_weight's grad_reduce_group is refused."""
+    inp = G.small_inputs(N=256, H=128, V=640, seed=29, n_ign=40, w_std=0.1)
+    h = G.bf16_tensor(inp.hidden_bits).requires_grad_(True)
+    w = G.bf16_tensor(inp.weight_bits).requires_grad_(True)
+    y = G.labels_tensor(inp.labels)
+    n_global = 1000  # e.g. this micro-batch is one of several
+    mod = flce.FusedLinearCrossEntropy(ignore_index=IGN, reduction="sum")
+    loss = mod(h.view(2, 128, 128), y.view(2, 128), w, num_label_tokens=n_global)
+    loss.backward()
+    rf = oracle.forward(inp.hidden, inp.weight, inp.labels, IGN, 0.0, "sum")
+    rb = oracle.backward(inp.hidden, inp.weight, inp.labels, IGN, 0.0, "sum",
+                         grad_scale=1.0 / n_global)
+    G.check_loss(loss.item(), rf["loss"] / n_global)
+    assert int(mod.num_tokens) == rf["num_tokens"]
+    assert G.rel_l2(h.grad.float().cpu().numpy().reshape(256, 128), rb["d_hidden"]) < 5e-3
+    assert G.rel_l2(w.grad.float().cpu().numpy(), rb["d_weight"]) < 5e-3
+    # 'mean' ignores it
+    mean = flce.FusedLinearCrossEntropy(ignore_index=IGN, reduction="mean")
+    a = mean(h, y, w, num_label_tokens=n_global).item()
+    b = mean(h, y, w).item()
+    assert a == b
+    with pytest.raises(NotImplementedError):
+        mod(h, y, w, grad_reduce_group=object())
