@@ -141,6 +141,9 @@ flce_status flce_forward_ex(const void* hidden, const void* weight, const int64_
  *                (bf16[N*H] with FLCE_DHIDDEN_BF16)
  *   d_weight     device float[V*H]  overwritten, or accumulated into
  *                (bf16[V*H] with FLCE_DWEIGHT_BF16)
+ *                Either may be NULL: that gradient is then not computed (a
+ *                frozen LM head needs no dWeight GEMM: a third of the work);
+ *                at least one must be given.
  *   flags        any OR of FLCE_ACCUMULATE_DHIDDEN, FLCE_ACCUMULATE_DWEIGHT,
  *                FLCE_DHIDDEN_BF16, FLCE_DWEIGHT_BF16, or 0.
  * A bf16 output is computed in fp32 scratch inside the workspace (size it with

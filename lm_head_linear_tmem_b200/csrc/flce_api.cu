@@ -574,6 +574,8 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
                           int32_t flags, void* ws, cudaStream_t st) {
   const bool acc_dh = (flags & FLCE_ACCUMULATE_DHIDDEN) != 0;
   const bool acc_dw = (flags & FLCE_ACCUMULATE_DWEIGHT) != 0;
+  const bool want_dh = d_hidden != nullptr;  // a NULL output is not computed
+  const bool want_dw = d_weight != nullptr;
   const Chunking ck = chunking(N, V);
   const BwdLayout BL = bwd_layout(N, H, V);
   char* w = static_cast<char*>(ws);
@@ -654,7 +656,7 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
         gather_rows_kernel<<<n, 256, 0, st>>>(
             static_cast<const uint4*>(hidden), static_cast<int>(H / 8), n, perm, n_valid_c,
             static_cast<uint4*>(hidden_c), reinterpret_cast<float4*>(d_hidden),
-            static_cast<int>(H / 4), acc_dh ? 0 : 1);
+            static_cast<int>(H / 4), (want_dh && !acc_dh) ? 1 : 0);
       });
     if (e != cudaSuccess) return cuda_fail(e);
     hid = hidden_c;
@@ -670,8 +672,10 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
       !make_map(&t_hid_mn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hid, H, N, H * 2, 64, BK) ||
       !make_map(&t_w_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, weight, H, V, H * 2, BK, b_box_rows()) ||
       !make_map(&t_w_mn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, weight, H, V, H * 2, 64, BK) ||
-      !make_map(&t_dh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d_hidden, H, N, H * 4, 32, 32) ||
-      !make_map(&t_dw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d_weight, H, V, H * 4, 32, 32))
+      (want_dh &&
+       !make_map(&t_dh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d_hidden, H, N, H * 4, 32, 32)) ||
+      (want_dw &&
+       !make_map(&t_dw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d_weight, H, V, H * 4, 32, 32)))
     return FLCE_ERR_CUDA;
   // H a multiple of 64: the MN-major hidden and weight operands use the 3-D view
   // (FLCE_MN3D=0: every MN-major operand uses the 2-D view; read at every call)
@@ -784,19 +788,20 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
 
       const GemmProblem ph{&t_g_k, &t_w_mn, &t_dh, rows, gh};
       const GemmProblem pw{&t_g_mn, &t_hid_mn, &t_dw, cols, gw};
-      if (bwd_fuse_dhdw()) {
+      if (want_dh && want_dw && bwd_fuse_dhdw()) {
         // 2) + 3) in one launch: the dWeight tiles fill the dHidden grid's last wave
         e = run_gemm<StoreEpi, false, true, true, true>(d, kSlotDh, kBwdDhDw, ph, eh, &pw, ew, st);
       } else {
-        e = run_gemm<StoreEpi, false, true>(d, kSlotDh, kBwdDhDw, ph, eh, nullptr, eh, st);
-        if (e == cudaSuccess)
+        if (want_dh)
+          e = run_gemm<StoreEpi, false, true>(d, kSlotDh, kBwdDhDw, ph, eh, nullptr, eh, st);
+        if (want_dw && e == cudaSuccess)
           e = run_gemm<StoreEpi, true, true>(d, kSlotDw, kBwdDhDw, pw, ew, nullptr, ew, st);
       }
       if (e != cudaSuccess) return cuda_fail(e);
     }
   }
 
-  if (compact) {
+  if (compact && want_dw) {
     // dWeight's exact label term, per label run (dHidden's was added above).
     float* part = reinterpret_cast<float*>(w + BL.part);
     const dim3 grid(static_cast<unsigned>((N + kFixSeg - 1) / kFixSeg),
@@ -833,7 +838,7 @@ flce_status backward_fp32(DevInfo* d, const void* hidden, const void* weight,
   if (e != cudaSuccess) return cuda_fail(e);
   e = set_smem_attr(d, 2 * kSlotSimtDw, simt_dw_kernel, 2 * kSimtMaxH * 4 + kSimtThreads * 4);
   if (e != cudaSuccess) return cuda_fail(e);
-  if (n > 0) {
+  if (n > 0 && d_hidden != nullptr) {
     e = launch(kSimt, st, [&] {
       simt_dh_kernel<<<n, kSimtThreads, sh_dh, st>>>(
           static_cast<const float*>(hidden), static_cast<const float*>(weight), labels, lse, n, h,
@@ -841,6 +846,7 @@ flce_status backward_fp32(DevInfo* d, const void* hidden, const void* weight,
     });
     if (e != cudaSuccess) return cuda_fail(e);
   }
+  if (d_weight == nullptr) return FLCE_OK;
   e = launch(kSimt, st, [&] {
     simt_dw_kernel<<<v, kSimtThreads, sh_dw, st>>>(
         static_cast<const float*>(hidden), static_cast<const float*>(weight), labels, lse, n, h, v,
@@ -920,7 +926,8 @@ flce_status flce_backward(const void* hidden, const void* weight, const int64_t*
   if (s != FLCE_OK) return s;
   const GradScratch gs = grad_scratch(N, H, V, dtype == FLCE_BF16, flags);
   if (workspace_bytes < gs.end) return FLCE_ERR_WORKSPACE;
-  if (d_weight == nullptr || (N > 0 && (d_hidden == nullptr || lse == nullptr)))
+  // a NULL d_hidden or d_weight is not computed; one of them must be given
+  if ((d_hidden == nullptr && d_weight == nullptr) || (N > 0 && lse == nullptr))
     return FLCE_ERR_ARG;
   if (!aligned16(d_hidden) || !aligned16(d_weight)) return FLCE_ERR_ARG;
   if (!(grad_scale == grad_scale) || grad_scale == INFINITY || grad_scale == -INFINITY)
@@ -932,7 +939,7 @@ flce_status flce_backward(const void* hidden, const void* weight, const int64_t*
   cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(unsigned int), st);  // status word
   if (e != cudaSuccess) return cuda_fail(e);
   if (N == 0) {
-    if (flags & FLCE_ACCUMULATE_DWEIGHT) return FLCE_OK;  // adds nothing
+    if (d_weight == nullptr || (flags & FLCE_ACCUMULATE_DWEIGHT)) return FLCE_OK;  // adds nothing
     const size_t elem = (flags & FLCE_DWEIGHT_BF16) ? 2 : sizeof(float);  // +0.0 in both
     e = cudaMemsetAsync(d_weight, 0, static_cast<size_t>(V) * H * elem, st);
     return e == cudaSuccess ? FLCE_OK : cuda_fail(e);
@@ -940,8 +947,10 @@ flce_status flce_backward(const void* hidden, const void* weight, const int64_t*
   // bf16 outputs: the gradient is computed into fp32 scratch (overwritten, not
   // accumulated) and rounded once into the caller's buffer afterwards.
   char* wsb = static_cast<char*>(workspace);
-  float* dh32 = (flags & FLCE_DHIDDEN_BF16) ? reinterpret_cast<float*>(wsb + gs.dh) : d_hidden;
-  float* dw32 = (flags & FLCE_DWEIGHT_BF16) ? reinterpret_cast<float*>(wsb + gs.dw) : d_weight;
+  float* dh32 = (d_hidden != nullptr && (flags & FLCE_DHIDDEN_BF16))
+                    ? reinterpret_cast<float*>(wsb + gs.dh) : d_hidden;
+  float* dw32 = (d_weight != nullptr && (flags & FLCE_DWEIGHT_BF16))
+                    ? reinterpret_cast<float*>(wsb + gs.dw) : d_weight;
   int32_t inner = flags & (FLCE_ACCUMULATE_DHIDDEN | FLCE_ACCUMULATE_DWEIGHT);
   if (flags & FLCE_DHIDDEN_BF16) inner &= ~FLCE_ACCUMULATE_DHIDDEN;
   if (flags & FLCE_DWEIGHT_BF16) inner &= ~FLCE_ACCUMULATE_DWEIGHT;
@@ -980,7 +989,7 @@ flce_status flce_backward(const void* hidden, const void* weight, const int64_t*
                {FLCE_DWEIGHT_BF16, FLCE_ACCUMULATE_DWEIGHT, dw32, d_weight,
                 static_cast<size_t>(V) * H}};
   for (const auto& o : outs) {
-    if (!(flags & o.flag)) continue;
+    if (!(flags & o.flag) || o.dst == nullptr) continue;
     const unsigned blocks = static_cast<unsigned>(
         std::min<size_t>((o.n / 8 + 255) / 256 + 1, static_cast<size_t>(d->sms) * 8));
     e = launch(kHelper, st, [&] {

@@ -122,18 +122,26 @@ def backward(hidden: torch.Tensor, weight: torch.Tensor, labels: torch.Tensor,
              d_hidden: Optional[torch.Tensor] = None, d_weight: Optional[torch.Tensor] = None,
              accumulate_d_hidden: bool = False, accumulate_d_weight: bool = False,
              grad_dtype: torch.dtype = torch.float32,
-             check_status: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+             compute_d_hidden: bool = True, compute_d_weight: bool = True,
+             check_status: bool = False) -> Tuple[Optional[torch.Tensor], Optional[torch.Tensor]]:
     """dHidden [N, H] and dWeight [V, H], float32 or bfloat16 (the dtype of a
     given d_hidden / d_weight, else `grad_dtype`).  A bf16 gradient is
     computed in fp32 and rounded once.  With accumulate_* the gradient is
     added into the given d_hidden / d_weight instead of overwriting them (e.g.
-    over the micro-batches of one optimizer step)."""
+    over the micro-batches of one optimizer step).  compute_d_weight=False
+    (a frozen LM head) or compute_d_hidden=False skips that gradient's GEMM
+    and returns None in its place."""
     h2, w, y = _prep(hidden, weight, labels)
     N, H = h2.shape
     V = w.shape[0]
     dev = h2.device
     if grad_dtype not in (torch.float32, torch.bfloat16):
         raise TypeError("grad_dtype must be float32 or bfloat16")
+    if not (compute_d_hidden or compute_d_weight):
+        raise ValueError("nothing to compute: both gradients are switched off")
+    if (accumulate_d_hidden and not compute_d_hidden) or (accumulate_d_weight and
+                                                          not compute_d_weight):
+        raise ValueError("cannot accumulate a gradient that is not computed")
     for name, t, acc, shape in (("d_hidden", d_hidden, accumulate_d_hidden, (N, H)),
                                 ("d_weight", d_weight, accumulate_d_weight, (V, H))):
         if acc and t is None:
@@ -143,14 +151,20 @@ def backward(hidden: torch.Tensor, weight: torch.Tensor, labels: torch.Tensor,
                               or not t.is_contiguous() or t.device != dev):
             raise ValueError(f"{name} must be a contiguous float32 or bfloat16 {list(shape)} "
                              f"tensor on {dev}")
-    if d_hidden is None:
+    if not compute_d_hidden:
+        d_hidden = None
+    elif d_hidden is None:
         d_hidden = torch.empty((N, H), dtype=grad_dtype, device=dev)
-    if d_weight is None:
+    if not compute_d_weight:
+        d_weight = None
+    elif d_weight is None:
         d_weight = torch.empty((V, H), dtype=grad_dtype, device=dev)
     flags = ((_native.ACCUMULATE_DHIDDEN if accumulate_d_hidden else 0)
              | (_native.ACCUMULATE_DWEIGHT if accumulate_d_weight else 0)
-             | (_native.DHIDDEN_BF16 if d_hidden.dtype == torch.bfloat16 else 0)
-             | (_native.DWEIGHT_BF16 if d_weight.dtype == torch.bfloat16 else 0))
+             | (_native.DHIDDEN_BF16 if d_hidden is not None
+                and d_hidden.dtype == torch.bfloat16 else 0)
+             | (_native.DWEIGHT_BF16 if d_weight is not None
+                and d_weight.dtype == torch.bfloat16 else 0))
     if workspace is None:
         workspace = alloc_workspace(N, H, V, h2.dtype, dev, flags)
     if grad_output is not None:
@@ -185,13 +199,19 @@ class _FlceFunction(torch.autograd.Function):
     def backward(ctx, grad_loss, _grad_ntok):
         hidden, weight, labels, lse = ctx.saved_tensors
         ignore_index, softcap, reduction, grad_scale, hshape = ctx.cfg
-        # gradients in the parameters' own dtype (bf16 rounded once from fp32)
-        dh = torch.empty(hshape, dtype=hidden.dtype, device=hidden.device).view(-1, hshape[-1])
-        dw = torch.empty(weight.shape, dtype=weight.dtype, device=weight.device)
+        # gradients in the parameters' own dtype (bf16 rounded once from fp32),
+        # and only those autograd asks for (a frozen LM head skips dWeight)
+        need_dh, need_dw = ctx.needs_input_grad[0], ctx.needs_input_grad[1]
+        if not (need_dh or need_dw):
+            return (None,) * 8
+        dh = (torch.empty(hshape, dtype=hidden.dtype, device=hidden.device)
+              .view(-1, hshape[-1]) if need_dh else None)
+        dw = torch.empty(weight.shape, dtype=weight.dtype, device=weight.device) \
+            if need_dw else None
         backward(hidden, weight, labels, lse, grad_output=grad_loss, grad_scale=grad_scale,
                  ignore_index=ignore_index, softcap=softcap, reduction=reduction,
-                 d_hidden=dh, d_weight=dw)
-        return dh.view(hshape), dw, None, None, None, None, None, None
+                 d_hidden=dh, d_weight=dw, compute_d_hidden=need_dh, compute_d_weight=need_dw)
+        return (dh.view(hshape) if need_dh else None), dw, None, None, None, None, None, None
 
 
 def fused_linear_cross_entropy(hidden, weight, labels, ignore_index: int = -100,

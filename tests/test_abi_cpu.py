@@ -104,6 +104,9 @@ def test_argument_errors_are_synchronous(lib):
     bad_flags = lib.flce_backward(FAKE, FAKE, FAKE, FAKE, 64, 64, 512, -100, 0.0, 0, 0, None,
                                   1.0, None, FAKE, FAKE, 16, FAKE, wsb, None)
     assert bad_flags == ARG
+    no_outputs = lib.flce_backward(FAKE, FAKE, FAKE, FAKE, 64, 64, 512, -100, 0.0, 0, 0, None,
+                                   1.0, None, None, None, 0, FAKE, wsb, None)
+    assert no_outputs == ARG
     # bf16 gradient outputs need the larger workspace of flce_workspace_bytes_ex
     for flags in (4, 8, 12):
         assert lib.flce_backward(FAKE, FAKE, FAKE, FAKE, 64, 64, 512, -100, 0.0, 0, 0, None,

@@ -419,3 +419,32 @@ def test_module_num_label_tokens():
     assert a == b
     with pytest.raises(NotImplementedError):
         mod(h, y, w, grad_reduce_group=object())
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_optional_gradients(dtype):
+    """A NULL output skips its gradient (a frozen LM head needs no dWeight GEMM); the
+    other one is bit-identical to a full backward."""
+    if dtype == "bf16":
+        inp = G.small_inputs(N=2100, H=192, V=4500, seed=30, n_ign=300, w_std=0.1)
+        h, W = G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits)
+    else:
+        inp = G.small_inputs(N=200, H=64, V=700, seed=30, n_ign=20, w_std=0.1)
+        h, W = G.f32_tensor(inp.hidden_raw), G.f32_tensor(inp.weight_raw)
+    y = G.labels_tensor(inp.labels)
+    with G.chunks(*SMALL_CHUNKS):
+        f = flce.forward(h, W, y, softcap=3.0, check_status=True)
+        args = dict(softcap=3.0, grad_scale=0.4, check_status=True)
+        dh, dw = flce.backward(h, W, y, f.lse, **args)
+        only_dh, none_w = flce.backward(h, W, y, f.lse, compute_d_weight=False, **args)
+        none_h, only_dw = flce.backward(h, W, y, f.lse, compute_d_hidden=False, **args)
+        torch.cuda.synchronize()
+    assert none_w is None and none_h is None
+    assert torch.equal(only_dh, dh) and torch.equal(only_dw, dw)
+    if dtype == "bf16":  # autograd with a frozen LM head asks for dHidden alone
+        hh = h.clone().requires_grad_(True)
+        loss = flce.FusedLinearCrossEntropy(logit_softcapping=3.0)(hh, y, W)
+        loss.backward()
+        assert W.grad is None
+        assert torch.equal(hh.grad, (dh / 0.4).to(torch.bfloat16)) or \
+            G.rel_l2(hh.grad.float().cpu().numpy(), dh.cpu().numpy() / 0.4) < 5e-3
