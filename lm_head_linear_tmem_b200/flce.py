@@ -6,14 +6,16 @@ outputs and the workspace with torch, and passes raw device pointers and the
 current CUDA stream.  There is no CPU or PyTorch fallback.
 
 API (names follow the pages):
-  forward(hidden, weight, labels, ignore_index=-100, softcap=0.0, reduction='sum')
-      -> FlceForward(loss, num_tokens, lse)
+  forward(hidden, weight, labels, ignore_index=-100, softcap=0.0, reduction='sum',
+          loss_scale=1.0) -> FlceForward(loss, num_tokens, lse)
   backward(hidden, weight, labels, lse, grad_output=None, grad_scale=1.0, ...)
-      -> (d_hidden, d_weight)
+      -> (d_hidden, d_weight), fp32 or bf16, optionally accumulated into given
+         buffers, either one skippable
   FusedLinearCrossEntropy(ignore_index=-100, logit_softcapping=0, reduction='sum')
-      an nn.Module whose forward(hidden_states, labels, lm_weight) returns the
-      loss and records `num_tokens` ('sum': non-ignored count, 'mean': 0), as
-      the NeMo AutoModel linear_ce API and modelscope/twinkle PR #335 specify.
+      an nn.Module whose forward(hidden_states, labels, lm_weight,
+      num_label_tokens=None, grad_reduce_group=None) returns the loss and
+      records `num_tokens` ('sum': non-ignored count, 'mean': 0), as the NeMo
+      AutoModel linear_ce API and modelscope/twinkle PR #335 specify.
 """
 from __future__ import annotations
 
