@@ -52,9 +52,15 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["own", "reference"], default="own")
     p.add_argument("--workload", default=WORKLOAD)
-    p.add_argument("--cpu-sample-tokens", type=int, default=256)
+    p.add_argument("--cpu-sample-tokens", type=int, default=1536)
+    p.add_argument("--cpu-full", action="store_true",
+                   help="time the float64 oracle's forward+backward on the whole workload "
+                        "on the host cores (minutes; no GPU) and print one JSON line")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=None)
+    p.add_argument("--option", action="append", default=[], metavar="NAME=VALUE",
+                   help="set a library option (flce_set_option) for this run, e.g. "
+                        "grad_tile_n=256; may be repeated")
     return p.parse_args()
 
 
@@ -144,12 +150,52 @@ def blas_threads():
     return os.cpu_count() or 1
 
 
+CPU_FULL = os.path.join(ROOT, "profiles", "cpu_oracle_full_{}.json")
+
+
+def cpu_full_record(workload):
+    """The committed record of `bench.py --cpu-full` for this workload, if any."""
+    path = CPU_FULL.format(workload)
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        return json.load(f)
+
+
 def cpu_baseline(inp, w, tokens):
     W64 = inp.weight.astype(np.float64)
     secs = oracle_step_sample(inp, w, tokens, W64)
-    return {"value": tokens / secs, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": f"float64 numpy oracle fwd+bwd on the first {tokens} tokens of "
-                      f"{w.name} (H={w.H}, V={w.V}), {secs:.2f} s"}
+    out = {"value": tokens / secs, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+           "sample": f"float64 numpy oracle fwd+bwd on the first {tokens} tokens of "
+                     f"{w.name} (H={w.H}, V={w.V}), {secs:.2f} s",
+           "value_is": "the sampled rate, measured in this run"}
+    full = cpu_full_record(w.name)
+    if full is not None:
+        out["full_problem"] = {k: full[k] for k in ("wall_s", "tokens_per_s", "cores", "tokens",
+                                                    "command") if k in full}
+        out["full_problem"]["measured"] = "separately, by the command given (not in this run)"
+    return out
+
+
+def run_cpu_full(args):
+    """--cpu-full: the oracle's forward and backward over the whole workload, timed
+    once on the host cores (the float64 baseline at full size)."""
+    import oracle  # test infrastructure: the CPU baseline is the oracle itself
+    w = fi.WORKLOADS[args.workload]
+    inp = fi.make_inputs(w)
+    h = inp.hidden.astype(np.float64)
+    W64 = inp.weight.astype(np.float64)
+    t0 = time.perf_counter()
+    f = oracle.forward(h, W64, inp.labels, fi.IGNORE_INDEX, w.softcap, w.reduction)
+    t1 = time.perf_counter()
+    oracle.backward(h, W64, inp.labels, fi.IGNORE_INDEX, w.softcap, w.reduction)
+    t2 = time.perf_counter()
+    line = {"kind": "oracle", "workload": w.name, "tokens": w.N, "hidden": w.H, "vocab": w.V,
+            "forward_s": t1 - t0, "backward_s": t2 - t1, "wall_s": t2 - t0,
+            "tokens_per_s": w.N / (t2 - t0), "cores": blas_threads(),
+            "cpu_count": os.cpu_count(), "loss": f["loss"],
+            "command": f"python bench.py --cpu-full --workload {w.name}"}
+    print(json.dumps(line), flush=True)
 
 
 def run_reference(args, rank):
@@ -232,6 +278,10 @@ def run_own(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     lib = _native.load()
+    for kv in args.option:
+        name, val = kv.split("=")
+        _native.set_option(name, int(val))
+    options = {name: _native.get_option(name) for name in _native.OPTIONS}
     w = fi.WORKLOADS[args.workload]
     inp = fi.make_inputs(w)
     N, H, V = w.N, w.H, w.V
@@ -369,9 +419,9 @@ def run_own(args, rank, world, local_rank):
     flops_step = w.flops_per_step
     # Work the kernels execute: the forward covers every row; the backward GEMMs
     # cover the non-ignored rows only (rows with ignore_index have exactly zero
-    # gradient and are compacted away) unless FLCE_BWD_COMPACT=0.
+    # gradient and are compacted away) unless the bwd_compact option is off.
     n_valid = int((inp.labels != fi.IGNORE_INDEX).sum())
-    compact = os.environ.get("FLCE_BWD_COMPACT", "1") != "0"
+    compact = _native.get_option("bwd_compact") != 0
     n_bwd = n_valid if compact else N
     executed_step = 2.0 * N * H * V + 6.0 * n_bwd * H * V
     # the dominant kernel (largest device time) and its roofline
@@ -430,6 +480,7 @@ def run_own(args, rank, world, local_rank):
         "gemm_roofline": gemm_roofline,
         "kernels": kinds,
         "kernels_region_ms_per_step": ms_prof / args.steps,
+        "library_options": options,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
@@ -447,6 +498,10 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.cpu_full:
+        if rank == 0:
+            run_cpu_full(args)
+        return
     if args.impl == "reference":
         run_reference(args, rank)
         return

@@ -92,6 +92,39 @@ typedef enum flce_reduction { FLCE_SUM = 0, FLCE_MEAN = 1 } flce_reduction;
 
 typedef enum flce_dtype { FLCE_BF16 = 0, FLCE_FP32 = 1 } flce_dtype;
 
+/* Library options (flce_set_option).  They are process-wide, apply to every
+ * device, and keep their value until set again; every call reads them once,
+ * when it starts.  None changes the result beyond fp32 summation order: they
+ * select between equivalent schedules (for measurements and tests) and set
+ * limits.  Nothing else (no environment variable) changes what the library
+ * runs.  Defaults in brackets. */
+typedef enum flce_option {
+  FLCE_OPT_CTA_GROUP = 0,       /* [2] tensor-core tiles of CTA pairs (256 rows); 1: single CTAs (128 rows) */
+  FLCE_OPT_BWD_COMPACT = 1,     /* [1] the backward leaves ignored rows out of its GEMMs; 0: keeps every row
+                                   (and then also skips the exact fp32 label-term correction) */
+  FLCE_OPT_BWD_FUSE = 2,        /* [1] dHidden and dWeight GEMMs of a backward chunk share one launch; 0: two */
+  FLCE_OPT_MN3D = 3,            /* [1] MN-major operands load through 3-D chunk views; 0: 2-D views */
+  FLCE_OPT_CHUNK_TOKENS = 4,    /* [8192] token rows of a backward chunk (256 .. 2^20, rounded up to 256) */
+  FLCE_OPT_CHUNK_VOCAB = 5,     /* [16384] vocab columns of a backward chunk (256 .. 2^20, rounded up to 256);
+                                   the dZ block of the workspace is chunk_tokens x chunk_vocab bf16, so
+                                   flce_workspace_bytes must be called with the same chunk options as the
+                                   calls that use the workspace */
+  FLCE_OPT_WAIT_TIMEOUT_MS = 6, /* [1000] limit of every bounded wait inside a kernel (10 .. 60000) */
+  FLCE_OPT_GRAD_TILE_N = 7,     /* [512] columns of a dHidden / dWeight tile: 512 or 256 (512 needs CTA pairs;
+                                   with FLCE_OPT_CTA_GROUP = 1 tiles are 256 wide) */
+  FLCE_OPT_DZ_TILE_N = 8,       /* [256] columns of a backward dZ tile: 256 or 512 (as above) */
+  FLCE_OPT_FWD_TILE_N = 9,      /* [256] columns of a forward tile: 256 or 512 (as above) */
+  FLCE_OPT_COUNT_ = 10          /* number of options (not an option) */
+} flce_option;
+
+/* Set option `option` to `value`.  FLCE_ERR_ARG for an unknown option or a
+ * value outside its range; the option is then unchanged. */
+flce_status flce_set_option(int32_t option, int64_t value);
+
+/* Current value of `option` into *value.  FLCE_ERR_ARG for an unknown option
+ * or a NULL value. */
+flce_status flce_get_option(int32_t option, int64_t* value);
+
 /* Bytes of workspace that flce_forward / flce_backward need for this shape.
  * Returns 0 for invalid sizes.  Pure host computation. */
 size_t flce_workspace_bytes(int64_t N, int64_t H, int64_t V, int32_t dtype);
@@ -124,6 +157,25 @@ flce_status flce_forward_ex(const void* hidden, const void* weight, const int64_
                             int32_t reduction, int32_t dtype, float loss_scale, float* loss,
                             int64_t* num_tokens, float* lse, void* workspace,
                             size_t workspace_bytes, void* stream);
+
+/* flce_forward_ex with, in addition, the global number of label tokens that
+ * normalises a 'sum' loss (NeMo AutoModel linear_ce API, forward(
+ * num_label_tokens): the count of non-padding target tokens across the
+ * micro-batches and ranks that share one optimizer step).
+ *   num_label_tokens >= 0, 'sum': loss = loss_scale * (sum_i loss_i) /
+ *       max(num_label_tokens, 1), evaluated in float64 before the single
+ *       rounding to float32 (the max(., 1) clamp keeps a batch without target
+ *       tokens at 0, never NaN: inclusionAI/Ling-3.1-flash discussion #7, "Why
+ *       use num_items_in_batch for MTP?");
+ *   num_label_tokens < 0 (none given), or 'mean' (which divides by its own
+ *       count): as flce_forward_ex.
+ * num_tokens and lse are unchanged by either scale.  The matching backward is
+ * flce_backward_ex with the same num_label_tokens and grad_scale = loss_scale. */
+flce_status flce_forward_ex2(const void* hidden, const void* weight, const int64_t* labels,
+                             int64_t N, int64_t H, int64_t V, int64_t ignore_index, float softcap,
+                             int32_t reduction, int32_t dtype, float loss_scale,
+                             int64_t num_label_tokens, float* loss, int64_t* num_tokens,
+                             float* lse, void* workspace, size_t workspace_bytes, void* stream);
 
 /* flce_backward flags. */
 #define FLCE_ACCUMULATE_DHIDDEN 1 /* d_hidden += gradient (else overwritten) */
@@ -162,6 +214,19 @@ flce_status flce_backward(const void* hidden, const void* weight, const int64_t*
                           const float* grad_output, float grad_scale, const int64_t* num_valid,
                           float* d_hidden, float* d_weight, int32_t flags, void* workspace,
                           size_t workspace_bytes, void* stream);
+
+/* flce_backward for the loss of flce_forward_ex2: with num_label_tokens >= 0
+ * and 'sum', the gradient factor g is divided by max(num_label_tokens, 1)
+ * (computed in float64 with grad_scale, then rounded once to float32);
+ * num_label_tokens < 0 or 'mean': exactly flce_backward.  Every other argument
+ * as flce_backward. */
+flce_status flce_backward_ex(const void* hidden, const void* weight, const int64_t* labels,
+                             const float* lse, int64_t N, int64_t H, int64_t V,
+                             int64_t ignore_index, float softcap, int32_t reduction,
+                             int32_t dtype, const float* grad_output, float grad_scale,
+                             int64_t num_label_tokens, const int64_t* num_valid,
+                             float* d_hidden, float* d_weight, int32_t flags, void* workspace,
+                             size_t workspace_bytes, void* stream);
 
 /* Size of the library-owned device buffer behind flce_forward_noalloc. */
 #define FLCE_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)

@@ -11,9 +11,10 @@ from .flce import (  # noqa: F401
     FlceForward, FusedLinearCrossEntropy, alloc_workspace, backward, forward,
     fused_linear_cross_entropy, status, workspace_bytes,
 )
-from ._native import FlceError, load  # noqa: F401
+from ._native import FlceError, get_option, load, options, set_option  # noqa: F401
 
 __all__ = [
     "FlceForward", "FusedLinearCrossEntropy", "FlceError", "alloc_workspace", "backward",
-    "forward", "fused_linear_cross_entropy", "load", "status", "workspace_bytes",
+    "forward", "fused_linear_cross_entropy", "get_option", "load", "options", "set_option",
+    "status", "workspace_bytes",
 ]

@@ -4,6 +4,7 @@ Loading fails loudly: there is no CPU or PyTorch fallback for any FLCE step.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -28,6 +29,12 @@ BF16, FP32 = 0, 1
 ACCUMULATE_DHIDDEN, ACCUMULATE_DWEIGHT = 1, 2
 DHIDDEN_BF16, DWEIGHT_BF16 = 4, 8
 
+# flce_option values (include/flce.h)
+OPTIONS = {
+    "cta_group": 0, "bwd_compact": 1, "bwd_fuse": 2, "mn3d": 3, "chunk_tokens": 4,
+    "chunk_vocab": 5, "wait_timeout_ms": 6, "grad_tile_n": 7, "dz_tile_n": 8, "fwd_tile_n": 9,
+}
+
 # Every symbol include/flce.h declares, with its ctypes signature.
 SIGNATURES = {
     "flce_workspace_bytes": (c_size, [c_i64, c_i64, c_i64, c_i32]),
@@ -36,9 +43,16 @@ SIGNATURES = {
                              c_i32, c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),
     "flce_forward_ex": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32, c_i32,
                                 c_i32, c_f32, c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),
+    "flce_forward_ex2": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32, c_i32,
+                                 c_i32, c_f32, c_i64, c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),
     "flce_backward": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32,
                               c_i32, c_i32, c_vp, c_f32, c_vp, c_vp, c_vp, c_i32, c_vp, c_size,
                               c_vp]),
+    "flce_backward_ex": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32,
+                                 c_i32, c_i32, c_vp, c_f32, c_i64, c_vp, c_vp, c_vp, c_i32, c_vp,
+                                 c_size, c_vp]),
+    "flce_set_option": (c_i32, [c_i32, c_i64]),
+    "flce_get_option": (c_i32, [c_i32, ctypes.POINTER(c_i64)]),
     "flce_forward_noalloc": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_f32,
                                      c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "flce_get_status": (c_i32, [c_vp, c_vp]),
@@ -90,3 +104,28 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
 def check(status: int, where: str) -> None:
     if status != FLCE_OK:
         raise FlceError(status, where)
+
+
+def get_option(name: str) -> int:
+    """Current value of a library option (see flce_option in include/flce.h)."""
+    v = c_i64()
+    check(load().flce_get_option(OPTIONS[name], ctypes.byref(v)), f"flce_get_option({name})")
+    return int(v.value)
+
+
+def set_option(name: str, value: int) -> None:
+    """Set a process-wide library option (flce_set_option)."""
+    check(load().flce_set_option(OPTIONS[name], int(value)), f"flce_set_option({name}={value})")
+
+
+@contextlib.contextmanager
+def options(**values):
+    """Set library options for the duration of a `with` block, then restore them."""
+    old = {k: get_option(k) for k in values}
+    try:
+        for k, v in values.items():
+            set_option(k, v)
+        yield
+    finally:
+        for k, v in old.items():
+            set_option(k, v)

@@ -199,34 +199,84 @@ FwdLayout fwd_layout(int64_t N, int64_t V, bool bf16) {
   return L;
 }
 
+// ---------------------------------------------------------------- options
+// Process-wide settings (flce_set_option).  Every call takes one snapshot of
+// them at its start, so a concurrent flce_set_option never changes a call
+// half-way; flce_workspace_bytes and the calls that use the workspace must see
+// the same chunk sizes.
+struct OptSpec {
+  int64_t dflt, lo, hi;
+};
+constexpr int kNumOpts = FLCE_OPT_COUNT_;
+constexpr OptSpec kOptSpec[kNumOpts] = {
+    {2, 1, 2},                 // FLCE_OPT_CTA_GROUP
+    {1, 0, 1},                 // FLCE_OPT_BWD_COMPACT
+    {1, 0, 1},                 // FLCE_OPT_BWD_FUSE
+    {1, 0, 1},                 // FLCE_OPT_MN3D
+    {kChunkTokens, 256, 1 << 20},  // FLCE_OPT_CHUNK_TOKENS
+    {kChunkVocab, 256, 1 << 20},   // FLCE_OPT_CHUNK_VOCAB
+    {1000, 10, 60000},         // FLCE_OPT_WAIT_TIMEOUT_MS
+    {512, 256, 512},           // FLCE_OPT_GRAD_TILE_N
+    {256, 256, 512},           // FLCE_OPT_DZ_TILE_N
+    {256, 256, 512},           // FLCE_OPT_FWD_TILE_N
+};
+std::atomic<int64_t> g_opt[kNumOpts] = {
+    {kOptSpec[0].dflt}, {kOptSpec[1].dflt}, {kOptSpec[2].dflt}, {kOptSpec[3].dflt},
+    {kOptSpec[4].dflt}, {kOptSpec[5].dflt}, {kOptSpec[6].dflt}, {kOptSpec[7].dflt},
+    {kOptSpec[8].dflt}, {kOptSpec[9].dflt}};
+
+struct Opts {
+  int cta_group;          // 2: CTA pairs with 256-row tiles; 1: single CTAs, 128-row tiles
+  bool compact;           // backward leaves ignored rows out of its GEMMs
+  bool fuse;              // dHidden and dWeight GEMMs of a chunk share one launch
+  bool mn3d;              // MN-major operands load through 3-D chunk views
+  int64_t chunk_tokens;   // backward chunk (multiples of 256)
+  int64_t chunk_vocab;
+  unsigned long long timeout_ns;  // limit of every bounded wait inside a kernel
+  int grad_bn;            // columns of a dHidden / dWeight tile (512 needs CTA pairs)
+  int dz_bn;              // columns of a dZ tile
+  int fwd_bn;             // columns of a forward tile
+};
+
+Opts opts() {
+  Opts o;
+  o.cta_group = static_cast<int>(g_opt[FLCE_OPT_CTA_GROUP].load());
+  o.compact = g_opt[FLCE_OPT_BWD_COMPACT].load() != 0;
+  o.fuse = g_opt[FLCE_OPT_BWD_FUSE].load() != 0;
+  o.mn3d = g_opt[FLCE_OPT_MN3D].load() != 0;
+  o.chunk_tokens = align_up(static_cast<size_t>(g_opt[FLCE_OPT_CHUNK_TOKENS].load()), 256);
+  o.chunk_vocab = align_up(static_cast<size_t>(g_opt[FLCE_OPT_CHUNK_VOCAB].load()), 256);
+  o.timeout_ns = static_cast<unsigned long long>(g_opt[FLCE_OPT_WAIT_TIMEOUT_MS].load()) * 1000000ull;
+  o.grad_bn = (o.cta_group == 2) ? static_cast<int>(g_opt[FLCE_OPT_GRAD_TILE_N].load()) : 256;
+  o.dz_bn = (o.cta_group == 2) ? static_cast<int>(g_opt[FLCE_OPT_DZ_TILE_N].load()) : 256;
+  o.fwd_bn = (o.cta_group == 2) ? static_cast<int>(g_opt[FLCE_OPT_FWD_TILE_N].load()) : 256;
+  return o;
+}
+
+// Divisor of a 'sum' loss (and of its gradient) normalised by the global
+// number of label tokens: max(num_label_tokens, 1), the clamp that keeps an
+// all-ignored batch at 0 instead of NaN; 1 when no count is given (< 0) or for
+// 'mean', which divides by its own count.
+double label_token_divisor(int32_t reduction, int64_t num_label_tokens) {
+  if (reduction != FLCE_SUM || num_label_tokens < 0) return 1.0;
+  return static_cast<double>(num_label_tokens > 0 ? num_label_tokens : 1);
+}
+
 struct Chunking {
   int tc, vc;  // chunk sizes (tokens, vocab)
 };
 
-// FLCE_CHUNK_TOKENS / FLCE_CHUNK_VOCAB override the chunk sizes (rounded up to
-// a multiple of 256; read at every call, so flce_workspace_bytes and the
-// calls that use the workspace must see the same values).
-int64_t chunk_size(const char* env, int64_t dflt) {
-  const char* s = std::getenv(env);
-  if (s == nullptr) return dflt;
-  const long long v = std::atoll(s);
-  if (v <= 0) return dflt;
-  return align_up(std::min<int64_t>(v, int64_t{1} << 20), 256);
-}
-
-Chunking chunking(int64_t N, int64_t V) {
+Chunking chunking(const Opts& o, int64_t N, int64_t V) {
   Chunking c;
-  const int64_t kt = chunk_size("FLCE_CHUNK_TOKENS", kChunkTokens);
-  const int64_t kv = chunk_size("FLCE_CHUNK_VOCAB", kChunkVocab);
-  c.tc = static_cast<int>(std::min<int64_t>(kt, align_up(std::max<int64_t>(N, 1), BM)));
-  c.vc = static_cast<int>(std::min<int64_t>(kv, align_up(V, BN)));
+  c.tc = static_cast<int>(std::min<int64_t>(o.chunk_tokens, align_up(std::max<int64_t>(N, 1), BM)));
+  c.vc = static_cast<int>(std::min<int64_t>(o.chunk_vocab, align_up(V, BN)));
   return c;
 }
 
 // Backward GEMM launches of one call (at most three per chunk), each with its
 // own dynamic tile counter in the workspace.
-int64_t bwd_launches(int64_t N, int64_t V) {
-  const Chunking c = chunking(N, V);
+int64_t bwd_launches(const Opts& o, int64_t N, int64_t V) {
+  const Chunking c = chunking(o, N, V);
   return 3 * ((N + c.tc - 1) / c.tc) * ((V + c.vc - 1) / c.vc);
 }
 
@@ -240,13 +290,13 @@ struct BwdLayout {
       hist, resid, hidden_c, gblock, part, end;
 };
 
-BwdLayout bwd_layout(int64_t N, int64_t H, int64_t V) {
+BwdLayout bwd_layout(const Opts& o, int64_t N, int64_t H, int64_t V) {
   BwdLayout L{};
-  const Chunking c = chunking(N, V);
+  const Chunking c = chunking(o, N, V);
   const size_t nblk = static_cast<size_t>((N + kCompactThreads - 1) / kCompactThreads);
   size_t off = kHeaderBytes;
   L.counters = off;
-  off = align_up(off + 4 * static_cast<size_t>(bwd_launches(N, V)), 256);
+  off = align_up(off + 4 * static_cast<size_t>(bwd_launches(o, N, V)), 256);
   L.perm = off;
   off = align_up(off + 4 * static_cast<size_t>(N), 256);
   L.labels_c = off;
@@ -274,13 +324,13 @@ BwdLayout bwd_layout(int64_t N, int64_t H, int64_t V) {
   return L;
 }
 
-size_t bwd_bytes(int64_t N, int64_t H, int64_t V, bool bf16) {
+size_t bwd_bytes(const Opts& o, int64_t N, int64_t H, int64_t V, bool bf16) {
   if (!bf16) return kHeaderBytes;
-  return bwd_layout(N, H, V).end;
+  return bwd_layout(o, N, H, V).end;
 }
 
-size_t ws_bytes(int64_t N, int64_t H, int64_t V, bool bf16) {
-  return align_up(std::max(fwd_layout(N, V, bf16).end, bwd_bytes(N, H, V, bf16)), 256);
+size_t ws_bytes(const Opts& o, int64_t N, int64_t H, int64_t V, bool bf16) {
+  return align_up(std::max(fwd_layout(N, V, bf16).end, bwd_bytes(o, N, H, V, bf16)), 256);
 }
 
 // bf16 gradient outputs: fp32 scratch for dHidden and/or dWeight after the
@@ -292,9 +342,10 @@ struct GradScratch {
   size_t dh, dw, end;  // byte offsets (dh / dw meaningful only with their flag)
 };
 
-GradScratch grad_scratch(int64_t N, int64_t H, int64_t V, bool bf16, int32_t flags) {
+GradScratch grad_scratch(const Opts& o, int64_t N, int64_t H, int64_t V, bool bf16,
+                         int32_t flags) {
   GradScratch g{};
-  size_t off = align_up(ws_bytes(N, H, V, bf16), 256);
+  size_t off = align_up(ws_bytes(o, N, H, V, bf16), 256);
   g.dh = off;
   if (flags & FLCE_DHIDDEN_BF16) off = align_up(off + 4 * static_cast<size_t>(N) * H, 256);
   g.dw = off;
@@ -308,47 +359,13 @@ long long* ws_nvalid(void* ws) {
   return reinterpret_cast<long long*>(reinterpret_cast<char*>(ws) + 8);
 }
 
-// Tile shape of the tensor-core GEMMs: 2 = CTA pairs with 256 x 256 tiles
-// (default), 1 = single CTAs with 128 x 256 tiles.  FLCE_CTA_GROUP=1 selects
-// the latter (read at every call).
-int cta_group() {
-  const char* s = std::getenv("FLCE_CTA_GROUP");
-  return (s != nullptr && std::atoi(s) == 1) ? 1 : 2;
-}
-
-// Backward row compaction: token rows whose label is ignore_index are left out
-// of the backward GEMMs (default), or FLCE_BWD_COMPACT=0 keeps every row
-// (read at every call).
-bool bwd_compact() {
-  const char* s = std::getenv("FLCE_BWD_COMPACT");
-  return !(s != nullptr && std::atoi(s) == 0);
-}
-
-// Backward chunk schedule: the dHidden and dWeight GEMMs of a chunk share one
-// launch (default; tiles handed out dynamically, the long dHidden tiles
-// first), or FLCE_BWD_FUSE=0 gives each its own launch (read at every call).
-bool bwd_fuse_dhdw() {
-  const char* s = std::getenv("FLCE_BWD_FUSE");
-  return !(s != nullptr && std::atoi(s) == 0);
-}
-
-unsigned long long timeout_ns() {
-  static unsigned long long t = [] {
-    const char* s = std::getenv("FLCE_WAIT_TIMEOUT_MS");
-    long long ms = s ? std::atoll(s) : 1000;
-    if (ms < 10) ms = 10;
-    if (ms > 60000) ms = 60000;
-    return static_cast<unsigned long long>(ms) * 1000000ull;
-  }();
-  return t;
-}
 
 // ---------------------------------------------------------------- checks
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-flce_status check_common(const void* hidden, const void* weight, const int64_t* labels,
-                         int64_t N, int64_t H, int64_t V, float softcap, int32_t reduction,
-                         int32_t dtype, void* ws, size_t ws_size) {
+flce_status check_common(const Opts& o, const void* hidden, const void* weight,
+                         const int64_t* labels, int64_t N, int64_t H, int64_t V, float softcap,
+                         int32_t reduction, int32_t dtype, void* ws, size_t ws_size) {
   if (reduction != FLCE_SUM && reduction != FLCE_MEAN) return FLCE_ERR_ARG;
   if (dtype != FLCE_BF16 && dtype != FLCE_FP32) return FLCE_ERR_ARG;
   if (!(softcap >= 0.f) || !(softcap < INFINITY)) return FLCE_ERR_ARG;
@@ -360,7 +377,7 @@ flce_status check_common(const void* hidden, const void* weight, const int64_t* 
   if (!aligned16(hidden) || !aligned16(weight) || !aligned16(ws)) return FLCE_ERR_ARG;
   if ((reinterpret_cast<uintptr_t>(labels) & 7u) != 0) return FLCE_ERR_ARG;
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return FLCE_ERR_ARG;
-  if (ws_size < ws_bytes(N, H, V, dtype == FLCE_BF16)) return FLCE_ERR_WORKSPACE;
+  if (ws_size < ws_bytes(o, N, H, V, dtype == FLCE_BF16)) return FLCE_ERR_WORKSPACE;
   return FLCE_OK;
 }
 
@@ -369,7 +386,7 @@ std::mutex g_attr_mu;
 std::set<std::pair<int, const void*>> g_attr_done;
 
 template <class Kern>
-cudaError_t set_smem_attr(DevInfo*, int, Kern k, size_t bytes) {
+cudaError_t set_smem_attr(Kern k, size_t bytes) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -386,36 +403,38 @@ cudaError_t set_smem_attr(DevInfo*, int, Kern k, size_t bytes) {
   return e;
 }
 
-// Kernel instantiation slots for the shared-memory attribute cache (x2: CTA group).
-enum Slot { kSlotFwd = 0, kSlotFwdCap, kSlotDz, kSlotDzCap, kSlotDh, kSlotDw, kSlotSimtDh, kSlotSimtDw };
-
 // One GEMM of a launch: operand / output tensor maps, output rows M (tiled by
-// 128 * kCG) and the rest of its GemmArgs.
+// 128 * kCG), output columns Ncols (tiled by the launch's tile width) and the
+// rest of its GemmArgs.
 struct GemmProblem {
   const CUtensorMap* a;
   const CUtensorMap* b;
   const CUtensorMap* out;
   int64_t M;
+  int64_t Ncols;
   GemmArgs g;
 };
 
 // One tensor-core launch over one GEMM (p1 == nullptr) or two independent
 // GEMMs with the same epilogue.  kCG = 2 launches clusters of two CTAs.
-template <class Epi, int kCG, bool kAMn0, bool kBMn0, bool kAMn1, bool kBMn1>
-cudaError_t run_gemm_cg(DevInfo* d, int slot, int kind, const GemmProblem& p0,
+template <class Epi, int kCG, int kBN, bool kAMn0, bool kBMn0, bool kAMn1, bool kBMn1>
+cudaError_t run_gemm_cg(DevInfo* d, int kind, const GemmProblem& p0,
                         const typename Epi::Params& ep0, const GemmProblem* p1,
                         const typename Epi::Params& ep1, cudaStream_t st) {
-  using Cfg = TileCfg<kCG>;
-  auto k = tc_gemm_kernel<Epi, kCG, kAMn0, kBMn0, kAMn1, kBMn1>;
-  cudaError_t e = set_smem_attr(d, 2 * slot + (kCG - 1), k, Cfg::kSmemBytes);
+  using Cfg = TileCfg<kCG, kBN>;
+  auto k = tc_gemm_kernel<Epi, kCG, kBN, kAMn0, kBMn0, kAMn1, kBMn1>;
+  cudaError_t e = set_smem_attr(k, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
   GemmArgs g0 = p0.g;
   g0.m_tiles = static_cast<int>((p0.M + Cfg::kUnitRows - 1) / Cfg::kUnitRows);
+  g0.n_tiles = static_cast<int>((p0.Ncols + kBN - 1) / kBN);
   GemmArgs g1 = p1 ? p1->g : p0.g;
-  if (p1)
+  if (p1) {
     g1.m_tiles = static_cast<int>((p1->M + Cfg::kUnitRows - 1) / Cfg::kUnitRows);
-  else
+    g1.n_tiles = static_cast<int>((p1->Ncols + kBN - 1) / kBN);
+  } else {
     g1.m_tiles = g1.n_tiles = 0;
+  }
   const GemmProblem& q1 = p1 ? *p1 : p0;
   const int tiles = g0.m_tiles * g0.n_tiles + g1.m_tiles * g1.n_tiles;
   const int units = std::max(1, std::min(tiles, d->sms / kCG));
@@ -449,24 +468,28 @@ cudaError_t run_gemm_cg(DevInfo* d, int slot, int kind, const GemmProblem& p0,
   return le != cudaSuccess ? le : e2;
 }
 
+// The launch in the CTA group of `o` with tiles of `bn` columns (512 only
+// with CTA pairs; opts() guarantees it).
 template <class Epi, bool kAMn0, bool kBMn0, bool kAMn1 = false, bool kBMn1 = false>
-cudaError_t run_gemm(DevInfo* d, int slot, int kind, const GemmProblem& p0,
+cudaError_t run_gemm(DevInfo* d, const Opts& o, int bn, int kind, const GemmProblem& p0,
                      const typename Epi::Params& ep0, const GemmProblem* p1,
                      const typename Epi::Params& ep1, cudaStream_t st) {
-  if (cta_group() == 2)
-    return run_gemm_cg<Epi, 2, kAMn0, kBMn0, kAMn1, kBMn1>(d, slot, kind, p0, ep0, p1, ep1, st);
-  return run_gemm_cg<Epi, 1, kAMn0, kBMn0, kAMn1, kBMn1>(d, slot, kind, p0, ep0, p1, ep1, st);
+  if (o.cta_group == 1)
+    return run_gemm_cg<Epi, 1, 256, kAMn0, kBMn0, kAMn1, kBMn1>(d, kind, p0, ep0, p1, ep1, st);
+  if (bn == 512)
+    return run_gemm_cg<Epi, 2, 512, kAMn0, kBMn0, kAMn1, kBMn1>(d, kind, p0, ep0, p1, ep1, st);
+  return run_gemm_cg<Epi, 2, 256, kAMn0, kBMn0, kAMn1, kBMn1>(d, kind, p0, ep0, p1, ep1, st);
 }
 
-// Rows of B (K-major) one CTA stages per K-block.
-uint32_t b_box_rows() { return static_cast<uint32_t>(BN / cta_group()); }
+// Rows of B (K-major) one CTA stages per bank and K-block.
+uint32_t b_box_rows(const Opts& o) { return static_cast<uint32_t>(BN / o.cta_group); }
 
 // ---------------------------------------------------------------- forward
-flce_status forward_bf16(DevInfo* d, const void* hidden, const void* weight,
+flce_status forward_bf16(DevInfo* d, const Opts& o, const void* hidden, const void* weight,
                          const int64_t* labels, int64_t N, int64_t H, int64_t V,
                          int64_t ignore_index, float softcap, int32_t reduction,
-                         double loss_scale, float* loss, int64_t* num_tokens, float* lse,
-                         void* ws, cudaStream_t st) {
+                         double loss_scale, double loss_div, float* loss, int64_t* num_tokens,
+                         float* lse, void* ws, cudaStream_t st) {
   char* w = static_cast<char*>(ws);
   const FwdLayout L = fwd_layout(N, V, true);
   float* part_m = reinterpret_cast<float*>(w + L.part_m);
@@ -477,35 +500,34 @@ flce_status forward_bf16(DevInfo* d, const void* hidden, const void* weight,
 
   CUtensorMap ta, tb;
   if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hidden, H, N, H * 2, BK, BM) ||
-      !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, weight, H, V, H * 2, BK, b_box_rows()))
+      !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, weight, H, V, H * 2, BK, b_box_rows(o)))
     return FLCE_ERR_CUDA;
 
   GemmArgs g{};
-  g.n_tiles = static_cast<int>((V + BN - 1) / BN);
   g.k_blocks = static_cast<int>((H + BK - 1) / BK);
   g.group_m = kGroupM;
   g.a_off = 0;
   g.b_off = 0;
   g.status = ws_status(ws);
-  g.timeout_ns = timeout_ns();
+  g.timeout_ns = o.timeout_ns;
 
   cudaError_t e;
-  const GemmProblem prob{&ta, &tb, &ta, N, g};
+  const GemmProblem prob{&ta, &tb, &ta, N, V, g};
   if (softcap > 0.f) {
     FwdStatsEpi<true>::Params ep{labels, static_cast<int>(N), static_cast<int>(V), softcap,
                                  1.0f / softcap, part_m, part_s, label_logit};
-    e = run_gemm<FwdStatsEpi<true>, false, false>(d, kSlotFwdCap, kFwdGemm, prob, ep, nullptr,
+    e = run_gemm<FwdStatsEpi<true>, false, false>(d, o, o.fwd_bn, kFwdGemm, prob, ep, nullptr,
                                                   ep, st);
   } else {
     FwdStatsEpi<false>::Params ep{labels, static_cast<int>(N), static_cast<int>(V), 0.f, 0.f,
                                   part_m, part_s, label_logit};
-    e = run_gemm<FwdStatsEpi<false>, false, false>(d, kSlotFwd, kFwdGemm, prob, ep, nullptr, ep,
-                                                   st);
+    e = run_gemm<FwdStatsEpi<false>, false, false>(d, o, o.fwd_bn, kFwdGemm, prob, ep, nullptr,
+                                                   ep, st);
   }
   if (e != cudaSuccess) return cuda_fail(e);
 
   const int n = static_cast<int>(N);
-  const int n_vt = g.n_tiles;
+  const int n_vt = static_cast<int>((V + BN - 1) / BN);  // (m, s) partials per row
   e = launch(kFwdMerge, st, [&] {
     fwd_merge_kernel<<<(n + kMergeRows - 1) / kMergeRows, dim3(kMergeRows, kMergeSplit), 0, st>>>(
         part_m, part_s, n_vt, n, lse);
@@ -519,8 +541,8 @@ flce_status forward_bf16(DevInfo* d, const void* hidden, const void* weight,
   if (e != cudaSuccess) return cuda_fail(e);
   e = launch(kFwdMerge, st, [&] {
     finalize_kernel<<<1, kFinalThreads, 0, st>>>(block_loss, block_cnt, nblk,
-                                                 reduction == FLCE_MEAN, loss_scale, loss,
-                                                 num_tokens, ws_nvalid(ws));
+                                                 reduction == FLCE_MEAN, loss_scale, loss_div,
+                                                 loss, num_tokens, ws_nvalid(ws));
   });
   if (e != cudaSuccess) return cuda_fail(e);
   return FLCE_OK;
@@ -529,8 +551,8 @@ flce_status forward_bf16(DevInfo* d, const void* hidden, const void* weight,
 flce_status forward_fp32(DevInfo* d, const void* hidden, const void* weight,
                          const int64_t* labels, int64_t N, int64_t H, int64_t V,
                          int64_t ignore_index, float softcap, int32_t reduction,
-                         double loss_scale, float* loss, int64_t* num_tokens, float* lse,
-                         void* ws, cudaStream_t st) {
+                         double loss_scale, double loss_div, float* loss, int64_t* num_tokens,
+                         float* lse, void* ws, cudaStream_t st) {
   (void)d;
   char* w = static_cast<char*>(ws);
   const FwdLayout L = fwd_layout(N, V, false);
@@ -558,15 +580,15 @@ flce_status forward_fp32(DevInfo* d, const void* hidden, const void* weight,
   if (e != cudaSuccess) return cuda_fail(e);
   e = launch(kFwdMerge, st, [&] {
     finalize_kernel<<<1, kFinalThreads, 0, st>>>(block_loss, block_cnt, nblk,
-                                                 reduction == FLCE_MEAN, loss_scale, loss,
-                                                 num_tokens, ws_nvalid(ws));
+                                                 reduction == FLCE_MEAN, loss_scale, loss_div,
+                                                 loss, num_tokens, ws_nvalid(ws));
   });
   if (e != cudaSuccess) return cuda_fail(e);
   return FLCE_OK;
 }
 
 // ---------------------------------------------------------------- backward
-flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
+flce_status backward_bf16(DevInfo* d, const Opts& o, const void* hidden, const void* weight,
                           const int64_t* labels, const float* lse, int64_t N, int64_t H,
                           int64_t V, int64_t ignore_index, float softcap, int32_t reduction,
                           const float* grad_output, float grad_scale, const long long* n_valid,
@@ -576,21 +598,21 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
   const bool acc_dw = (flags & FLCE_ACCUMULATE_DWEIGHT) != 0;
   const bool want_dh = d_hidden != nullptr;  // a NULL output is not computed
   const bool want_dw = d_weight != nullptr;
-  const Chunking ck = chunking(N, V);
-  const BwdLayout BL = bwd_layout(N, H, V);
+  const Chunking ck = chunking(o, N, V);
+  const BwdLayout BL = bwd_layout(o, N, H, V);
   char* w = static_cast<char*>(ws);
   void* gbuf = w + BL.gblock;
   int* counters = reinterpret_cast<int*>(w + BL.counters);
   int next_counter = 0;
   {
-    const cudaError_t e = cudaMemsetAsync(counters, 0, 4 * bwd_launches(N, V), st);
+    const cudaError_t e = cudaMemsetAsync(counters, 0, 4 * bwd_launches(o, N, V), st);
     if (e != cudaSuccess) return cuda_fail(e);
   }
 
   // Row compaction: the GEMMs see the valid token rows first (compact hidden,
   // labels and lse), the device-side count bounds their token-row dimension,
   // and dHidden rows are scattered back through the permutation.
-  const bool compact = bwd_compact();
+  const bool compact = o.compact;
   const void* hid = hidden;
   const int64_t* lab = labels;
   const float* lsev = lse;
@@ -670,7 +692,7 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
   CUtensorMap t_hid_k, t_hid_mn, t_w_k, t_w_mn, t_dh, t_dw;
   if (!make_map(&t_hid_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hid, H, N, H * 2, BK, BM) ||
       !make_map(&t_hid_mn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hid, H, N, H * 2, 64, BK) ||
-      !make_map(&t_w_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, weight, H, V, H * 2, BK, b_box_rows()) ||
+      !make_map(&t_w_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, weight, H, V, H * 2, BK, b_box_rows(o)) ||
       !make_map(&t_w_mn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, weight, H, V, H * 2, 64, BK) ||
       (want_dh &&
        !make_map(&t_dh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d_hidden, H, N, H * 4, 32, 32)) ||
@@ -678,17 +700,15 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
        !make_map(&t_dw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d_weight, H, V, H * 4, 32, 32)))
     return FLCE_ERR_CUDA;
   // H a multiple of 64: the MN-major hidden and weight operands use the 3-D view
-  // (FLCE_MN3D=0: every MN-major operand uses the 2-D view; read at every call)
-  const char* mn3d_env = std::getenv("FLCE_MN3D");
-  const bool mn3d = !(mn3d_env != nullptr && std::atoi(mn3d_env) == 0);
+  // (FLCE_OPT_MN3D = 0: every MN-major operand uses the 2-D view)
+  const bool mn3d = o.mn3d;
   const bool h3d = mn3d && (H % 64 == 0);
   if (h3d && (!make_map_mn3d(&t_hid_mn, hid, H, N, H * 2) ||
               !make_map_mn3d(&t_w_mn, weight, H, V, H * 2)))
     return FLCE_ERR_CUDA;
 
-  const int n_tiles_h = static_cast<int>((H + BN - 1) / BN);
   const int k_blocks_h = static_cast<int>((H + BK - 1) / BK);
-  const unsigned long long tmo = timeout_ns();
+  const unsigned long long tmo = o.timeout_ns;
   const int mean = reduction == FLCE_MEAN;
 
   for (int64_t t0 = 0; t0 < N; t0 += ck.tc) {
@@ -711,7 +731,6 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
 
       // 1) dZ = f(hidden[t0:] . W[v0:]^T) -> bf16 block
       GemmArgs gz{};
-      gz.n_tiles = (cols + BN - 1) / BN;
       gz.k_blocks = k_blocks_h;
       gz.group_m = kGroupM;
       gz.a_off = static_cast<int>(t0);
@@ -727,22 +746,21 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
       // its main loop may start early, its first store waits for them
       gz.dep_wait = (t0 > 0 || v0 > 0) ? kDepBeforeStores : kDepNone;
       cudaError_t e;
-      const GemmProblem pz{&t_hid_k, &t_w_k, &t_g_store, rows, gz};
+      const GemmProblem pz{&t_hid_k, &t_w_k, &t_g_store, rows, cols, gz};
       if (softcap > 0.f) {
         DzEpi<true>::Params ep{lab,  lsev,    ignore_index, static_cast<int>(t0),
                                rows, static_cast<int>(v0), cols, softcap, 1.0f / softcap,
                                resid, V};
-        e = run_gemm<DzEpi<true>, false, false>(d, kSlotDzCap, kBwdDz, pz, ep, nullptr, ep, st);
+        e = run_gemm<DzEpi<true>, false, false>(d, o, o.dz_bn, kBwdDz, pz, ep, nullptr, ep, st);
       } else {
         DzEpi<false>::Params ep{lab,  lsev, ignore_index, static_cast<int>(t0), rows,
                                 static_cast<int>(v0), cols, 0.f, 0.f, resid, V};
-        e = run_gemm<DzEpi<false>, false, false>(d, kSlotDz, kBwdDz, pz, ep, nullptr, ep, st);
+        e = run_gemm<DzEpi<false>, false, false>(d, o, o.dz_bn, kBwdDz, pz, ep, nullptr, ep, st);
       }
       if (e != cudaSuccess) return cuda_fail(e);
 
       // 2) dHidden[t0:t0+rows] (+)= dZ . W[v0:v0+cols]
       GemmArgs gh{};
-      gh.n_tiles = n_tiles_h;
       gh.k_blocks = (cols + BK - 1) / BK;
       gh.group_m = kGroupMGrad;
       gh.a_off = 0;
@@ -766,7 +784,6 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
 
       // 3) dWeight[v0:v0+cols] (+)= dZ^T . hidden[t0:t0+rows]
       GemmArgs gw{};
-      gw.n_tiles = n_tiles_h;
       gw.k_blocks = (rows + BK - 1) / BK;
       gw.group_m = kGroupMGrad;
       gw.a_off = 0;
@@ -786,16 +803,17 @@ flce_status backward_bf16(DevInfo* d, const void* hidden, const void* weight,
                           static_cast<int>(V), grad_output, grad_scale, n_valid, mean,
                           nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0};
 
-      const GemmProblem ph{&t_g_k, &t_w_mn, &t_dh, rows, gh};
-      const GemmProblem pw{&t_g_mn, &t_hid_mn, &t_dw, cols, gw};
-      if (want_dh && want_dw && bwd_fuse_dhdw()) {
+      const GemmProblem ph{&t_g_k, &t_w_mn, &t_dh, rows, H, gh};
+      const GemmProblem pw{&t_g_mn, &t_hid_mn, &t_dw, cols, H, gw};
+      const int gbn = o.grad_bn;
+      if (want_dh && want_dw && o.fuse) {
         // 2) + 3) in one launch: the dWeight tiles fill the dHidden grid's last wave
-        e = run_gemm<StoreEpi, false, true, true, true>(d, kSlotDh, kBwdDhDw, ph, eh, &pw, ew, st);
+        e = run_gemm<StoreEpi, false, true, true, true>(d, o, gbn, kBwdDhDw, ph, eh, &pw, ew, st);
       } else {
         if (want_dh)
-          e = run_gemm<StoreEpi, false, true>(d, kSlotDh, kBwdDhDw, ph, eh, nullptr, eh, st);
+          e = run_gemm<StoreEpi, false, true>(d, o, gbn, kBwdDhDw, ph, eh, nullptr, eh, st);
         if (want_dw && e == cudaSuccess)
-          e = run_gemm<StoreEpi, true, true>(d, kSlotDw, kBwdDhDw, pw, ew, nullptr, ew, st);
+          e = run_gemm<StoreEpi, true, true>(d, o, gbn, kBwdDhDw, pw, ew, nullptr, ew, st);
       }
       if (e != cudaSuccess) return cuda_fail(e);
     }
@@ -834,9 +852,10 @@ flce_status backward_fp32(DevInfo* d, const void* hidden, const void* weight,
   const int mean = reduction == FLCE_MEAN;
   const size_t sh_dh = (2 * static_cast<size_t>(h) + kSimtChunk) * sizeof(float);
   const size_t sh_dw = (2 * static_cast<size_t>(h) + kSimtThreads) * sizeof(float);
-  cudaError_t e = set_smem_attr(d, 2 * kSlotSimtDh, simt_dh_kernel, 2 * kSimtMaxH * 4 + kSimtChunk * 4);
+  (void)d;
+  cudaError_t e = set_smem_attr(simt_dh_kernel, 2 * kSimtMaxH * 4 + kSimtChunk * 4);
   if (e != cudaSuccess) return cuda_fail(e);
-  e = set_smem_attr(d, 2 * kSlotSimtDw, simt_dw_kernel, 2 * kSimtMaxH * 4 + kSimtThreads * 4);
+  e = set_smem_attr(simt_dw_kernel, 2 * kSimtMaxH * 4 + kSimtThreads * 4);
   if (e != cudaSuccess) return cuda_fail(e);
   if (n > 0 && d_hidden != nullptr) {
     e = launch(kSimt, st, [&] {
@@ -866,21 +885,22 @@ extern "C" {
 size_t flce_workspace_bytes(int64_t N, int64_t H, int64_t V, int32_t dtype) {
   if (N < 0 || V < 1 || H < 8 || N > kMaxDim || V > kMaxDim) return 0;
   if (dtype != FLCE_BF16 && dtype != FLCE_FP32) return 0;
-  return ws_bytes(N, H, V, dtype == FLCE_BF16);
+  return ws_bytes(opts(), N, H, V, dtype == FLCE_BF16);
 }
 
 size_t flce_workspace_bytes_ex(int64_t N, int64_t H, int64_t V, int32_t dtype, int32_t flags) {
   if ((flags & ~kAllBwdFlags) != 0) return 0;
   if (flce_workspace_bytes(N, H, V, dtype) == 0) return 0;
-  return grad_scratch(N, H, V, dtype == FLCE_BF16, flags).end;
+  return grad_scratch(opts(), N, H, V, dtype == FLCE_BF16, flags).end;
 }
 
 flce_status flce_forward(const void* hidden, const void* weight, const int64_t* labels,
                          int64_t N, int64_t H, int64_t V, int64_t ignore_index, float softcap,
                          int32_t reduction, int32_t dtype, float* loss, int64_t* num_tokens,
                          float* lse, void* workspace, size_t workspace_bytes, void* stream) {
-  return flce_forward_ex(hidden, weight, labels, N, H, V, ignore_index, softcap, reduction, dtype,
-                         1.0f, loss, num_tokens, lse, workspace, workspace_bytes, stream);
+  return flce_forward_ex2(hidden, weight, labels, N, H, V, ignore_index, softcap, reduction,
+                          dtype, 1.0f, -1, loss, num_tokens, lse, workspace, workspace_bytes,
+                          stream);
 }
 
 flce_status flce_forward_ex(const void* hidden, const void* weight, const int64_t* labels,
@@ -888,9 +908,20 @@ flce_status flce_forward_ex(const void* hidden, const void* weight, const int64_
                             int32_t reduction, int32_t dtype, float loss_scale, float* loss,
                             int64_t* num_tokens, float* lse, void* workspace,
                             size_t workspace_bytes, void* stream) {
+  return flce_forward_ex2(hidden, weight, labels, N, H, V, ignore_index, softcap, reduction,
+                          dtype, loss_scale, -1, loss, num_tokens, lse, workspace,
+                          workspace_bytes, stream);
+}
+
+flce_status flce_forward_ex2(const void* hidden, const void* weight, const int64_t* labels,
+                             int64_t N, int64_t H, int64_t V, int64_t ignore_index, float softcap,
+                             int32_t reduction, int32_t dtype, float loss_scale,
+                             int64_t num_label_tokens, float* loss, int64_t* num_tokens,
+                             float* lse, void* workspace, size_t workspace_bytes, void* stream) {
   if (!(loss_scale == loss_scale) || loss_scale == INFINITY || loss_scale == -INFINITY)
     return FLCE_ERR_ARG;
-  flce_status s = check_common(hidden, weight, labels, N, H, V, softcap, reduction, dtype,
+  const Opts o = opts();
+  flce_status s = check_common(o, hidden, weight, labels, N, H, V, softcap, reduction, dtype,
                                workspace, workspace_bytes);
   if (s != FLCE_OK) return s;
   if (loss == nullptr || num_tokens == nullptr || (N > 0 && lse == nullptr)) return FLCE_ERR_ARG;
@@ -907,11 +938,12 @@ flce_status flce_forward_ex(const void* hidden, const void* weight, const int64_
       return cuda_fail(e);
     return FLCE_OK;
   }
+  const double div = label_token_divisor(reduction, num_label_tokens);
   if (dtype == FLCE_BF16)
-    return forward_bf16(d, hidden, weight, labels, N, H, V, ignore_index, softcap, reduction,
-                        loss_scale, loss, num_tokens, lse, workspace, st);
+    return forward_bf16(d, o, hidden, weight, labels, N, H, V, ignore_index, softcap, reduction,
+                        loss_scale, div, loss, num_tokens, lse, workspace, st);
   return forward_fp32(d, hidden, weight, labels, N, H, V, ignore_index, softcap, reduction,
-                      loss_scale, loss, num_tokens, lse, workspace, st);
+                      loss_scale, div, loss, num_tokens, lse, workspace, st);
 }
 
 flce_status flce_backward(const void* hidden, const void* weight, const int64_t* labels,
@@ -920,11 +952,24 @@ flce_status flce_backward(const void* hidden, const void* weight, const int64_t*
                           const float* grad_output, float grad_scale, const int64_t* num_valid,
                           float* d_hidden, float* d_weight, int32_t flags, void* workspace,
                           size_t workspace_bytes, void* stream) {
+  return flce_backward_ex(hidden, weight, labels, lse, N, H, V, ignore_index, softcap, reduction,
+                          dtype, grad_output, grad_scale, -1, num_valid, d_hidden, d_weight,
+                          flags, workspace, workspace_bytes, stream);
+}
+
+flce_status flce_backward_ex(const void* hidden, const void* weight, const int64_t* labels,
+                             const float* lse, int64_t N, int64_t H, int64_t V,
+                             int64_t ignore_index, float softcap, int32_t reduction,
+                             int32_t dtype, const float* grad_output, float grad_scale,
+                             int64_t num_label_tokens, const int64_t* num_valid,
+                             float* d_hidden, float* d_weight, int32_t flags, void* workspace,
+                             size_t workspace_bytes, void* stream) {
   if ((flags & ~kAllBwdFlags) != 0) return FLCE_ERR_ARG;
-  flce_status s = check_common(hidden, weight, labels, N, H, V, softcap, reduction, dtype,
+  const Opts o = opts();
+  flce_status s = check_common(o, hidden, weight, labels, N, H, V, softcap, reduction, dtype,
                                workspace, workspace_bytes);
   if (s != FLCE_OK) return s;
-  const GradScratch gs = grad_scratch(N, H, V, dtype == FLCE_BF16, flags);
+  const GradScratch gs = grad_scratch(o, N, H, V, dtype == FLCE_BF16, flags);
   if (workspace_bytes < gs.end) return FLCE_ERR_WORKSPACE;
   // a NULL d_hidden or d_weight is not computed; one of them must be given
   if ((d_hidden == nullptr && d_weight == nullptr) || (N > 0 && lse == nullptr))
@@ -932,6 +977,10 @@ flce_status flce_backward(const void* hidden, const void* weight, const int64_t*
   if (!aligned16(d_hidden) || !aligned16(d_weight)) return FLCE_ERR_ARG;
   if (!(grad_scale == grad_scale) || grad_scale == INFINITY || grad_scale == -INFINITY)
     return FLCE_ERR_ARG;
+  // the gradient of a 'sum' loss normalised by max(num_label_tokens, 1)
+  const float gscale =
+      static_cast<float>(static_cast<double>(grad_scale) /
+                         label_token_divisor(reduction, num_label_tokens));
   DevInfo* d = nullptr;
   s = device_info(&d);
   if (s != FLCE_OK) return s;
@@ -954,7 +1003,8 @@ flce_status flce_backward(const void* hidden, const void* weight, const int64_t*
   int32_t inner = flags & (FLCE_ACCUMULATE_DHIDDEN | FLCE_ACCUMULATE_DWEIGHT);
   if (flags & FLCE_DHIDDEN_BF16) inner &= ~FLCE_ACCUMULATE_DHIDDEN;
   if (flags & FLCE_DWEIGHT_BF16) inner &= ~FLCE_ACCUMULATE_DWEIGHT;
-  if (!(dtype == FLCE_BF16 && bwd_compact())) {  // the compaction checks the labels itself
+  const bool compacts = (dtype == FLCE_BF16 && o.compact);
+  if (!compacts) {  // the compaction checks the labels itself
     e = launch(kHelper, st, [&] {
       label_range_kernel<<<static_cast<unsigned>((N + 255) / 256), 256, 0, st>>>(
           labels, static_cast<int>(N), ignore_index, V, ws_status(workspace));
@@ -963,7 +1013,7 @@ flce_status flce_backward(const void* hidden, const void* weight, const int64_t*
   }
   const long long* nv = reinterpret_cast<const long long*>(num_valid);
   const bool own_count = (nv == nullptr);
-  if (nv == nullptr && !(dtype == FLCE_BF16 && bwd_compact())) {
+  if (nv == nullptr && !compacts) {
     long long* out = ws_nvalid(workspace);
     e = launch(kHelper, st, [&] {
       count_valid_kernel<<<1, kFinalThreads, 0, st>>>(labels, static_cast<int>(N), ignore_index,
@@ -973,11 +1023,12 @@ flce_status flce_backward(const void* hidden, const void* weight, const int64_t*
     nv = out;
   }
   if (dtype == FLCE_BF16)
-    s = backward_bf16(d, hidden, weight, labels, lse, N, H, V, ignore_index, softcap, reduction,
-                      grad_output, grad_scale, nv, own_count, dh32, dw32, inner, workspace, st);
+    s = backward_bf16(d, o, hidden, weight, labels, lse, N, H, V, ignore_index, softcap,
+                      reduction, grad_output, gscale, nv, own_count, dh32, dw32, inner, workspace,
+                      st);
   else
     s = backward_fp32(d, hidden, weight, labels, lse, N, H, V, ignore_index, softcap, reduction,
-                      grad_output, grad_scale, nv, dh32, dw32, inner, st);
+                      grad_output, gscale, nv, dh32, dw32, inner, st);
   if (s != FLCE_OK) return s;
   const struct {
     int32_t flag, acc;
@@ -988,16 +1039,33 @@ flce_status flce_backward(const void* hidden, const void* weight, const int64_t*
                 static_cast<size_t>(N) * H},
                {FLCE_DWEIGHT_BF16, FLCE_ACCUMULATE_DWEIGHT, dw32, d_weight,
                 static_cast<size_t>(V) * H}};
-  for (const auto& o : outs) {
-    if (!(flags & o.flag) || o.dst == nullptr) continue;
+  for (const auto& out : outs) {
+    if (!(flags & out.flag) || out.dst == nullptr) continue;
     const unsigned blocks = static_cast<unsigned>(
-        std::min<size_t>((o.n / 8 + 255) / 256 + 1, static_cast<size_t>(d->sms) * 8));
+        std::min<size_t>((out.n / 8 + 255) / 256 + 1, static_cast<size_t>(d->sms) * 8));
     e = launch(kHelper, st, [&] {
-      f32_to_bf16_kernel<<<blocks, 256, 0, st>>>(o.src, static_cast<__nv_bfloat16*>(o.dst), o.n,
-                                                 (flags & o.acc) ? 1 : 0);
+      f32_to_bf16_kernel<<<blocks, 256, 0, st>>>(out.src, static_cast<__nv_bfloat16*>(out.dst),
+                                                 out.n, (flags & out.acc) ? 1 : 0);
     });
     if (e != cudaSuccess) return cuda_fail(e);
   }
+  return FLCE_OK;
+}
+
+flce_status flce_set_option(int32_t option, int64_t value) {
+  if (option < 0 || option >= kNumOpts) return FLCE_ERR_ARG;
+  const OptSpec& sp = kOptSpec[option];
+  if (value < sp.lo || value > sp.hi) return FLCE_ERR_ARG;
+  if ((option == FLCE_OPT_GRAD_TILE_N || option == FLCE_OPT_DZ_TILE_N ||
+       option == FLCE_OPT_FWD_TILE_N) && value != 256 && value != 512)
+    return FLCE_ERR_ARG;
+  g_opt[option].store(value);
+  return FLCE_OK;
+}
+
+flce_status flce_get_option(int32_t option, int64_t* value) {
+  if (option < 0 || option >= kNumOpts || value == nullptr) return FLCE_ERR_ARG;
+  *value = g_opt[option].load();
   return FLCE_OK;
 }
 
@@ -1152,10 +1220,10 @@ extern "C" flce_status flce_forward_noalloc(const void* hidden, const void* weig
       return cuda_fail(e);
   } else {
     s = (dtype == FLCE_BF16)
-            ? forward_bf16(d, hidden, weight, labels, N, H, V, ignore_index, softcap, reduction,
-                           1.0, loss, num_tokens, lse, ws, st)
+            ? forward_bf16(d, opts(), hidden, weight, labels, N, H, V, ignore_index, softcap,
+                           reduction, 1.0, 1.0, loss, num_tokens, lse, ws, st)
             : forward_fp32(d, hidden, weight, labels, N, H, V, ignore_index, softcap, reduction,
-                           1.0, loss, num_tokens, lse, ws, st);
+                           1.0, 1.0, loss, num_tokens, lse, ws, st);
     if (s != FLCE_OK) return s;
   }
   if (status != nullptr) {

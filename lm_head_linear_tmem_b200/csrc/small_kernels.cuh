@@ -95,11 +95,13 @@ __global__ void __launch_bounds__(kLossThreads)
 }
 
 // One block: fixed-order float64 sum of the block partials, then the
-// reduction contract: 'sum' -> (sum, n); 'mean' -> (sum / max(n,1), 0).
+// reduction contract: 'sum' -> (sum, n); 'mean' -> (sum / max(n,1), 0).  The
+// returned loss is also multiplied by loss_scale and divided by loss_div (a
+// 'sum' loss normalised by a global token count), in float64.
 __global__ void __launch_bounds__(kFinalThreads)
     finalize_kernel(const double* __restrict__ block_loss, const long long* __restrict__ block_cnt,
-                    int nblk, int mean, double loss_scale, float* loss, int64_t* num_tokens,
-                    long long* n_valid_out) {
+                    int nblk, int mean, double loss_scale, double loss_div, float* loss,
+                    int64_t* num_tokens, long long* n_valid_out) {
   __shared__ double sl[kFinalThreads];
   __shared__ long long sc[kFinalThreads];
   const int t = threadIdx.x;
@@ -123,10 +125,11 @@ __global__ void __launch_bounds__(kFinalThreads)
     const long long n = sc[0];
     const double total = sl[0];
     if (mean) {
-      loss[0] = static_cast<float>(total / static_cast<double>(n > 0 ? n : 1) * loss_scale);
+      loss[0] = static_cast<float>(total / static_cast<double>(n > 0 ? n : 1) * loss_scale /
+                                   loss_div);
       num_tokens[0] = 0;
     } else {
-      loss[0] = static_cast<float>(total * loss_scale);
+      loss[0] = static_cast<float>(total * loss_scale / loss_div);
       num_tokens[0] = n;
     }
     if (n_valid_out != nullptr) *n_valid_out = n;

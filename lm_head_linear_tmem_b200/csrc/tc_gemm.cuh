@@ -3,21 +3,29 @@
 // One CTA per SM (192 threads, ~225 KB shared memory, all 512 TMEM columns).
 // Warp roles:
 //   warp 0  TMA producer   (one thread): K-blocks of A and B into a stage ring
-//   warp 1  MMA issuer     (one thread): tcgen05.mma K=16 steps, fp32 in TMEM;
-//                                        two 256-column accumulators so the
-//                                        epilogue of tile i overlaps the MMAs of i+1
+//   warp 1  MMA issuer     (one thread): tcgen05.mma K=16 steps, fp32 in TMEM
 //   warps 2-5 epilogue     (128 threads, thread = accumulator row): tcgen05.ld
 //                                        then an operation-specific epilogue
-// Two tile shapes (template parameter kCG, the CTA group):
-//   kCG = 1  one CTA computes a 128 x 256 tile (tcgen05.mma.cta_group::1,
-//            M=128 N=256), 4 stages of 48 KiB;
-//   kCG = 2  a cluster of two CTAs computes a 256 x 256 tile with one
+// Tile shapes (template parameters kCG, the CTA group, and kBN, the columns of
+// a tile):
+//   kCG = 1, kBN = 256  one CTA computes a 128 x 256 tile
+//            (tcgen05.mma.cta_group::1, M=128 N=256), 4 stages of 48 KiB;
+//   kCG = 2, kBN = 256  a cluster of two CTAs computes a 256 x 256 tile with one
 //            tcgen05.mma.cta_group::2 (M=256 N=256) issued by the pair's
 //            leader: each CTA stages its own 128 rows of A and 128 rows of B
 //            (32 KiB a stage, 6 stages) and holds its own 128 x 256
 //            accumulator rows in TMEM, so each SM moves half the operand bytes
-//            per FLOP of the 1-CTA shape.
-// K-block 64 (one 128-byte swizzle row of bf16).
+//            per FLOP of the 1-CTA shape (64 B per clock at the MMA rate);
+//   kCG = 2, kBN = 512  the pair computes a 256 x 512 tile as two M=256 N=256
+//            MMAs per K step that share the A operand: each CTA stages 128
+//            rows of A and 2 x 128 rows of B (48 KiB a stage, 4 stages), 48 B
+//            per clock at the MMA rate.  The accumulator fills all 512 TMEM
+//            columns; the epilogue drains it as two 256-column banks, and the
+//            next tile's MMAs start on bank 0 (for up to kStages - 1 K-blocks,
+//            whose stages stay held) while bank 1 is still being drained.
+// TMEM is treated as two banks of 256 columns.  A 256-column tile uses one
+// bank (tiles alternate, so the epilogue of one overlaps the MMAs of the next);
+// a 512-column tile uses both.  K-block 64 (one 128-byte swizzle row of bf16).
 //
 // Operands may be K-major (row-major [rows, K], the usual "TN" GEMM) or
 // MN-major (row-major [K, rows]); both are staged with 128-byte swizzle and
@@ -51,15 +59,20 @@ constexpr int kStagingPerWarp = 2 * kStagingBuf;  // double buffered
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
 
-template <int kCG>
+template <int kCG, int kBN = 256>
 struct TileCfg {
-  static constexpr int kBRows = BN / kCG;  // B rows (N index) staged by one CTA
+  static_assert(kBN == 256 || (kBN == 512 && kCG == 2), "512-column tiles need CTA pairs");
+  static constexpr int kBanks = kBN / BN;          // 256-column TMEM banks of one tile
+  static constexpr int kBankRows = BN / kCG;       // B rows of one bank staged by one CTA
+  static constexpr int kBankBytes = kBankRows * BK * 2;
+  static constexpr int kBRows = kBanks * kBankRows;  // B rows (N index) staged by one CTA
   static constexpr int kBBytes = kBRows * BK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = kCG == 1 ? 4 : 6;
+  static constexpr int kStages = (kCG == 1 || kBN == 512) ? 4 : 6;
   static constexpr int kUnitRows = BM * kCG;  // output rows of one tile
   static constexpr size_t kSmemBytes =
       1024 + static_cast<size_t>(kStages) * kStageBytes + kEpiWarps * kStagingPerWarp;
+  static_assert(kSmemBytes <= 227 * 1024 - 512, "shared memory");
 };
 
 constexpr int kRing = 8;  // tile indices in flight between the fetcher and the other roles
@@ -72,7 +85,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 struct GemmArgs {
   int m_tiles;    // tiles of kUnitRows output rows
-  int n_tiles;    // tiles of BN output columns
+  int n_tiles;    // tiles of kBN output columns
   int k_blocks;
   int group_m;    // tiles are walked in groups of group_m row-tiles (L2 reuse)
   int a_off;      // added to A's outer (row) TMA coordinate
@@ -157,12 +170,16 @@ struct FwdStatsEpi {
     float* label_logit;  // [N]
   };
 
-  __device__ static void tile(const Params& p, const GemmArgs&, int m_base, int nb,
+  __device__ static void tile(const Params& p, const GemmArgs&, int m_base, int col0,
                               uint32_t taddr, int q, int lane, uint8_t*, const CUtensorMap*,
                               uint32_t tempty, int&, bool) {
+    if (col0 >= p.V) {  // the second bank of a 512-column tile past the vocabulary
+      release_tmem(tempty, lane);
+      return;
+    }
     const int row = m_base + q * 32 + lane;
     const bool row_ok = row < p.N;
-    const int col0 = nb * BN;
+    const int nb = col0 / BN;
     int y_local = -1;
     if (row_ok) {
       const int64_t y = p.labels[row];
@@ -233,12 +250,12 @@ struct DzEpi {
     int64_t v_total;   // V: a label outside [0, V) counts as ignored
   };
 
-  __device__ static void tile(const Params& p, const GemmArgs&, int m_base, int nb,
+  __device__ static void tile(const Params& p, const GemmArgs&, int m_base, int col0,
                               uint32_t taddr, int q, int lane, uint8_t* stg,
                               const CUtensorMap* out, uint32_t tempty, int& nstore, bool) {
     // 64-column chunks whose store box starts inside the block (warp-uniform)
     const int y0 = m_base + q * 32;
-    const int rem = p.cols - nb * BN;
+    const int rem = p.cols - col0;
     const int nch = (y0 >= p.rows || rem <= 0) ? 0 : min(BN / 64, (rem + 63) / 64);
     if (nch == 0) {
       release_tmem(tempty, lane);
@@ -252,7 +269,7 @@ struct DzEpi {
       const int row = p.t0 + row_l;
       const int64_t y = p.labels[row];
       valid = (y != p.ignore_index) && y >= 0 && y < p.v_total;
-      const int64_t c0 = static_cast<int64_t>(p.v0) + static_cast<int64_t>(nb) * BN;
+      const int64_t c0 = static_cast<int64_t>(p.v0) + col0;
       if (valid && y >= c0 && y < c0 + BN) y_local = static_cast<int>(y - c0);
       lse2 = p.lse[row] * kLog2e;
     }
@@ -296,7 +313,7 @@ struct DzEpi {
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        tma_store_2d(out, stg_u32 + b * kStagingBuf, nb * BN + c2 * 64, y0);
+        tma_store_2d(out, stg_u32 + b * kStagingBuf, col0 + c2 * 64, y0);
         bulk_commit_group();
       }
       ++nstore;
@@ -342,7 +359,7 @@ struct StoreEpi {
     return g;
   }
 
-  __device__ static void tile(const Params& p, const GemmArgs&, int m_base, int nb,
+  __device__ static void tile(const Params& p, const GemmArgs&, int m_base, int col0,
                               uint32_t taddr, int q, int lane, uint8_t* stg,
                               const CUtensorMap* out, uint32_t tempty, int& nstore,
                               bool empty) {
@@ -350,24 +367,26 @@ struct StoreEpi {
     int y_end = p.y_limit;
     if (p.row_map != nullptr) y_end = static_cast<int>(min(static_cast<long long>(y_end), *p.rows_valid));
     // 32-column chunks whose store box starts inside the output (warp-uniform)
-    const int rem = p.x_limit - nb * BN;
+    const int rem = p.x_limit - col0;
     const int nch = (y >= y_end || rem <= 0) ? 0 : min(BN / 32, (rem + 31) / 32);
     if (nch == 0) {
       release_tmem(tempty, lane);
       return;
     }
-    const float g = empty ? 0.0f : grad_factor(p);  // an empty K range contributes zeros
+    // An empty K range contributes zeros: the accumulator was never written, so
+    // its stale contents are not read (0 * stale could be NaN).
+    const float g = empty ? 0.0f : grad_factor(p);
     if (p.row_map != nullptr) {
       const int r = y + lane;
       const bool live = r < y_end;
-      float* dst = p.out_ptr + static_cast<size_t>(live ? p.row_map[r] : 0) * p.ld + nb * BN;
+      float* dst = p.out_ptr + static_cast<size_t>(live ? p.row_map[r] : 0) * p.ld + col0;
       float cfix = 0.f;
       const __nv_bfloat16* wrow = nullptr;
-      if (p.fix_resid != nullptr && live) {
+      if (p.fix_resid != nullptr && live && !empty) {
         const int64_t yl = p.fix_labels[r];
         if (yl >= 0 && yl < p.fix_v) {
-          cfix = grad_factor(p) * p.fix_resid[r];
-          wrow = p.fix_w + static_cast<size_t>(yl) * p.x_limit + nb * BN;
+          cfix = g * p.fix_resid[r];
+          wrow = p.fix_w + static_cast<size_t>(yl) * p.x_limit + col0;
         }
       }
 #pragma unroll 1
@@ -376,10 +395,14 @@ struct StoreEpi {
         tmem_ld_x32(taddr + c * 32, v);
         tmem_ld_wait();
         if (c == nch - 1) release_tmem(tempty, lane);
+        if (empty) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = 0u;
+        }
         if (live) {
 #pragma unroll
           for (int j4 = 0; j4 < 8; ++j4) {
-            if (nb * BN + c * 32 + 4 * j4 >= p.x_limit) break;  // x_limit is a multiple of 4
+            if (col0 + c * 32 + 4 * j4 >= p.x_limit) break;  // x_limit is a multiple of 4
             float4 o = make_float4(__uint_as_float(v[4 * j4]) * g, __uint_as_float(v[4 * j4 + 1]) * g,
                                    __uint_as_float(v[4 * j4 + 2]) * g, __uint_as_float(v[4 * j4 + 3]) * g);
             float4* d4 = reinterpret_cast<float4*>(dst + c * 32) + j4;
@@ -413,7 +436,7 @@ struct StoreEpi {
       tmem_ld_wait();
       if (c == nch - 1) release_tmem(tempty, lane);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * g);
+      for (int j = 0; j < 32; ++j) r[j] = empty ? 0u : __float_as_uint(__uint_as_float(r[j]) * g);
       const int b = nstore & 1;  // see DzEpi
       if (lane == 0) bulk_wait_group_read<1>();
       __syncwarp();
@@ -421,7 +444,7 @@ struct StoreEpi {
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        const int x = nb * BN + c * 32;
+        const int x = col0 + c * 32;
         if (p.reduce)
           tma_reduce_add_2d(out, stg_u32 + b * kStagingBuf, x, y);
         else
@@ -468,15 +491,20 @@ __device__ __forceinline__ void load_mn(uint32_t dst, const CUtensorMap* map, ui
 // One launch runs the tiles of one GEMM, or of two independent GEMMs that
 // share the epilogue type (problem 0's tiles first, then problem 1's, so the
 // last wave of one is filled by the other).  Operand majors are per problem.
-template <class Epi, int kCG, bool kAMn0, bool kBMn0, bool kAMn1 = false, bool kBMn1 = false>
+template <class Epi, int kCG, int kBN, bool kAMn0, bool kBMn0, bool kAMn1 = false,
+          bool kBMn1 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                    const __grid_constant__ CUtensorMap tmOut0, const __grid_constant__ CUtensorMap tmA1,
                    const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmOut1,
                    const GemmArgs g0, const GemmArgs g1, const typename Epi::Params ep0,
                    const typename Epi::Params ep1) {
-  using Cfg = TileCfg<kCG>;
+  using Cfg = TileCfg<kCG, kBN>;
   constexpr int kStages = Cfg::kStages;
+  constexpr int kBanks = Cfg::kBanks;
+  // K-blocks of a 512-column tile issued on bank 0 alone while bank 1 still
+  // holds the previous tile (their stages stay held until bank 1 catches up)
+  constexpr int kStagger = kStages - 1;
   extern __shared__ uint8_t smem_dyn[];
   __shared__ __align__(8) uint64_t bar_full[kStages];
   __shared__ __align__(8) uint64_t bar_empty[kStages];
@@ -641,7 +669,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool a_mn = prob ? kAMn1 : kAMn0;
         const bool b_mn = prob ? kBMn1 : kBMn0;
         const int m_cta = mb * Cfg::kUnitRows + static_cast<int>(rank) * BM;
-        const int n_cta = nb * BN + static_cast<int>(rank) * Cfg::kBRows;
+        // bank h of the tile: B rows nb * kBN + h * BN + [rank * kBankRows, + kBankRows)
+        const int n_cta = nb * kBN + static_cast<int>(rank) * Cfg::kBankRows;
         for (int kb = 0; kb < g.k_blocks; ++kb) {
           if (!mbar_wait(smem_u32(&bar_empty[stage]), phase ^ 1u, abort_flag, g0.timeout_ns)) {
             ok = false;
@@ -663,10 +692,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             load_2d<kCG>(sa, mA, fb, kb * BK, g.a_off + m_cta);
           }
-          if (b_mn) {
-            load_mn<kCG>(sb, mB, fb, Cfg::kBRows, n_cta, g.b_off + kb * BK, g.b_mn3d != 0);
-          } else {
-            load_2d<kCG>(sb, mB, fb, kb * BK, g.b_off + n_cta);
+#pragma unroll
+          for (int h = 0; h < kBanks; ++h) {
+            const uint32_t sbh = sb + h * Cfg::kBankBytes;
+            if (b_mn) {
+              load_mn<kCG>(sbh, mB, fb, Cfg::kBankRows, n_cta + h * BN, g.b_off + kb * BK,
+                           g.b_mn3d != 0);
+            } else {
+              load_2d<kCG>(sbh, mB, fb, kb * BK, g.b_off + n_cta + h * BN);
+            }
           }
           issued_mask |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -697,6 +731,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool issued = false;
       int rslot = 0;
       uint32_t rph = 0;
+      // The 4 K=16 MMAs of one K-block of stage `st` with B part `part` of the
+      // stage (the tile's bank `part`) into TMEM bank `bank`; `first`: the
+      // K-block starts the accumulation.
+      auto mma_kblock = [&](uint32_t st, int part, uint32_t bank, bool first, uint32_t idesc,
+                            bool a_mn, bool b_mn) {
+        const uint32_t sa = smem_u32(smem + st * Cfg::kStageBytes);
+        const uint32_t sb = sa + kABytes + part * Cfg::kBankBytes;
+        const uint32_t d_tmem = tmem_base + bank * BN;
+#pragma unroll
+        for (int j = 0; j < BK / 16; ++j) {
+          const uint64_t ad = a_mn ? umma_desc_sw128(sa + j * 2048, 8192, 1024)
+                                   : umma_desc_sw128(sa + j * 32, 16, 1024);
+          const uint64_t bd = b_mn ? umma_desc_sw128(sb + j * 2048, 8192, 1024)
+                                   : umma_desc_sw128(sb + j * 32, 16, 1024);
+          const uint32_t accum = (!first || j > 0) ? 1u : 0u;
+          if constexpr (kCG == 1)
+            tc_mma_bf16(d_tmem, ad, bd, idesc, accum);
+          else
+            tc_mma_bf16_pair(d_tmem, ad, bd, idesc, accum);
+        }
+      };
+      auto commit_to = [&](uint64_t* bar) {
+        if constexpr (kCG == 1)
+          tc_commit(smem_u32(bar));
+        else
+          tc_commit_pair_mc(smem_u32(bar), 0x3);
+      };
+      auto next_stage = [&]() {
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      };
       for (;; ++it) {
         int tile;
         ok = ring_take(rslot, rph, false, tile);
@@ -710,49 +777,78 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t idesc = prob ? idesc1 : idesc0;
         const bool a_mn = prob ? kAMn1 : kAMn0;
         const bool b_mn = prob ? kBMn1 : kBMn0;
-        const uint32_t acc = it & 1;
-        const uint32_t aph = (it >> 1) & 1;
-        if (!mbar_wait(smem_u32(&bar_tempty[acc]), aph ^ 1u, abort_flag, g0.timeout_ns)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = 0; kb < k_blocks; ++kb) {
-          if (!mbar_wait(smem_u32(&bar_full[stage]), phase, abort_flag, g0.timeout_ns)) {
+        if constexpr (kBanks == 1) {
+          // tiles alternate between the two banks
+          const uint32_t acc = it & 1;
+          const uint32_t aph = (it >> 1) & 1;
+          if (!mbar_wait(smem_u32(&bar_tempty[acc]), aph ^ 1u, abort_flag, g0.timeout_ns)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * Cfg::kStageBytes);
-          const uint32_t sb = sa + kABytes;
-#pragma unroll
-          for (int j = 0; j < BK / 16; ++j) {
-            const uint64_t ad = a_mn ? umma_desc_sw128(sa + j * 2048, 8192, 1024)
-                                     : umma_desc_sw128(sa + j * 32, 16, 1024);
-            const uint64_t bd = b_mn ? umma_desc_sw128(sb + j * 2048, 8192, 1024)
-                                     : umma_desc_sw128(sb + j * 32, 16, 1024);
-            const uint32_t accum = (kb > 0 || j > 0) ? 1u : 0u;
-            if constexpr (kCG == 1)
-              tc_mma_bf16(d_tmem, ad, bd, idesc, accum);
-            else
-              tc_mma_bf16_pair(d_tmem, ad, bd, idesc, accum);
+          for (int kb = 0; kb < k_blocks; ++kb) {
+            if (!mbar_wait(smem_u32(&bar_full[stage]), phase, abort_flag, g0.timeout_ns)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            mma_kblock(stage, 0, acc, kb == 0, idesc, a_mn, b_mn);
+            issued = true;
+            commit_to(&bar_empty[stage]);
+            next_stage();
           }
-          issued = true;
-          if constexpr (kCG == 1)
-            tc_commit(smem_u32(&bar_empty[stage]));
-          else
-            tc_commit_pair_mc(smem_u32(&bar_empty[stage]), 0x3);
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1u;
+          if (!ok) break;
+          commit_to(&bar_tfull[acc]);
+        } else {
+          // one tile spans both banks.  Bank 0 starts as soon as the epilogue
+          // has drained it: its first d K-blocks run while bank 1 is still
+          // drained, their stages held; then bank 1 catches up on those stages
+          // and the rest of the K-blocks feed both banks.
+          const uint32_t aph = it & 1;
+          const int d = min(kStagger, k_blocks);
+          if (!mbar_wait(smem_u32(&bar_tempty[0]), aph ^ 1u, abort_flag, g0.timeout_ns)) {
+            ok = false;
+            break;
           }
+          tc_fence_after();
+          const uint32_t st0 = stage;
+          for (int kb = 0; kb < d; ++kb) {
+            if (!mbar_wait(smem_u32(&bar_full[stage]), phase, abort_flag, g0.timeout_ns)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            mma_kblock(stage, 0, 0, kb == 0, idesc, a_mn, b_mn);
+            issued = true;
+            next_stage();
+          }
+          if (!ok) break;
+          if (!mbar_wait(smem_u32(&bar_tempty[1]), aph ^ 1u, abort_flag, g0.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint32_t s1 = st0;
+          for (int kb = 0; kb < d; ++kb) {
+            mma_kblock(s1, 1, 1, kb == 0, idesc, a_mn, b_mn);
+            commit_to(&bar_empty[s1]);
+            s1 = (s1 + 1 == kStages) ? 0u : s1 + 1;
+          }
+          for (int kb = d; kb < k_blocks; ++kb) {
+            if (!mbar_wait(smem_u32(&bar_full[stage]), phase, abort_flag, g0.timeout_ns)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            mma_kblock(stage, 0, 0, false, idesc, a_mn, b_mn);
+            mma_kblock(stage, 1, 1, false, idesc, a_mn, b_mn);
+            issued = true;
+            commit_to(&bar_empty[stage]);
+            next_stage();
+          }
+          if (!ok) break;
+          commit_to(&bar_tfull[0]);
         }
-        if (!ok) break;
-        if constexpr (kCG == 1)
-          tc_commit(smem_u32(&bar_tfull[acc]));
-        else
-          tc_commit_pair_mc(smem_u32(&bar_tfull[acc]), 0x3);
       }
       if (!ok) {
         record_timeout(g0, abort_flag);
@@ -787,8 +883,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok || tile >= num_tiles) break;
       int prob, mb, nb;
       locate(tile, prob, mb, nb);
-      const uint32_t acc = it & 1;
-      const uint32_t aph = (it >> 1) & 1;
+      // the tile's first bank and the phase its full barrier completes
+      const uint32_t acc = (kBanks == 1) ? (it & 1) : 0u;
+      const uint32_t aph = (kBanks == 1) ? ((it >> 1) & 1) : (it & 1);
       bool w = mbar_wait(smem_u32(&bar_tfull[acc]), aph, abort_flag, g0.timeout_ns);
       w = __all_sync(0xffffffffu, w);
       if (!w) {
@@ -796,13 +893,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t taddr = tmem_base + acc * BN + (static_cast<uint32_t>(q * 32) << 16);
-      const uint32_t tempty_local = smem_u32(&bar_tempty[acc]);
-      const uint32_t tempty = (kCG == 1) ? tempty_local : mapa_shared(tempty_local, 0);
       const int m_base = mb * Cfg::kUnitRows + static_cast<int>(rank) * BM;
       const GemmArgs& ga = prob ? a1 : a0;
-      Epi::tile(prob ? ep1 : ep0, ga, m_base, nb, taddr, q, lane, stg, prob ? &tmOut1 : &tmOut0,
-                tempty, nstore, ga.k_blocks == 0);
+#pragma unroll 1
+      for (int h = 0; h < kBanks; ++h) {  // bank 0 first: the next tile starts on it
+        const uint32_t bank = acc + h;
+        const uint32_t taddr = tmem_base + bank * BN + (static_cast<uint32_t>(q * 32) << 16);
+        const uint32_t tempty_local = smem_u32(&bar_tempty[bank]);
+        const uint32_t tempty = (kCG == 1) ? tempty_local : mapa_shared(tempty_local, 0);
+        Epi::tile(prob ? ep1 : ep0, ga, m_base, nb * kBN + h * BN, taddr, q, lane, stg,
+                  prob ? &tmOut1 : &tmOut0, tempty, nstore, ga.k_blocks == 0);
+      }
     }
     if (lane == 0) {
       bulk_wait_group_all();

@@ -7,10 +7,13 @@ current CUDA stream.  There is no CPU or PyTorch fallback.
 
 API (names follow the pages):
   forward(hidden, weight, labels, ignore_index=-100, softcap=0.0, reduction='sum',
-          loss_scale=1.0) -> FlceForward(loss, num_tokens, lse)
-  backward(hidden, weight, labels, lse, grad_output=None, grad_scale=1.0, ...)
+          loss_scale=1.0, num_label_tokens=None) -> FlceForward(loss, num_tokens, lse)
+  backward(hidden, weight, labels, lse, grad_output=None, grad_scale=1.0,
+           num_label_tokens=None, ...)
       -> (d_hidden, d_weight), fp32 or bf16, optionally accumulated into given
          buffers, either one skippable
+  options(**values), set_option, get_option: the library's process-wide
+      settings (schedule switches and limits; see flce_option in flce.h)
   FusedLinearCrossEntropy(ignore_index=-100, logit_softcapping=0, reduction='sum')
       an nn.Module whose forward(hidden_states, labels, lm_weight,
       num_label_tokens=None, grad_reduce_group=None) returns the loss and
@@ -91,11 +94,24 @@ def status(workspace: torch.Tensor) -> int:
                                       ctypes.c_void_p(_stream(workspace.device))))
 
 
+def _count(num_label_tokens: Optional[int]) -> int:
+    """The C ABI's encoding of an optional global label-token count (-1: none)."""
+    if num_label_tokens is None:
+        return -1
+    n = int(num_label_tokens)
+    if n < 0:
+        raise ValueError("num_label_tokens must be >= 0")
+    return n
+
+
 def forward(hidden: torch.Tensor, weight: torch.Tensor, labels: torch.Tensor,
             ignore_index: int = -100, softcap: float = 0.0, reduction: str = "sum",
             workspace: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-            check_status: bool = False, loss_scale: float = 1.0) -> FlceForward:
-    """loss ('sum' or 'mean', times loss_scale), num_tokens and every row's lse."""
+            check_status: bool = False, loss_scale: float = 1.0,
+            num_label_tokens: Optional[int] = None) -> FlceForward:
+    """loss ('sum' or 'mean', times loss_scale), num_tokens and every row's lse.
+    With num_label_tokens, a 'sum' loss is normalised by that global count (the
+    library divides by max(num_label_tokens, 1))."""
     h2, w, y = _prep(hidden, weight, labels)
     N, H = h2.shape
     V = w.shape[0]
@@ -106,10 +122,11 @@ def forward(hidden: torch.Tensor, weight: torch.Tensor, labels: torch.Tensor,
     ntok = torch.empty((), dtype=torch.int64, device=dev)
     if lse is None:
         lse = torch.empty(N, dtype=torch.float32, device=dev)
-    st = _lib().flce_forward_ex(_ptr(h2), _ptr(w), _ptr(y), N, H, V, int(ignore_index),
-                                float(softcap), _REDUCTIONS[reduction], _DTYPES[h2.dtype],
-                                float(loss_scale), _ptr(loss), _ptr(ntok), _ptr(lse),
-                                _ptr(workspace), workspace.numel(), _stream(dev))
+    st = _lib().flce_forward_ex2(_ptr(h2), _ptr(w), _ptr(y), N, H, V, int(ignore_index),
+                                 float(softcap), _REDUCTIONS[reduction], _DTYPES[h2.dtype],
+                                 float(loss_scale), _count(num_label_tokens), _ptr(loss),
+                                 _ptr(ntok), _ptr(lse), _ptr(workspace), workspace.numel(),
+                                 _stream(dev))
     _native.check(st, "flce_forward")
     if check_status:
         _native.check(status(workspace), "flce_forward (device status)")
@@ -119,6 +136,7 @@ def forward(hidden: torch.Tensor, weight: torch.Tensor, labels: torch.Tensor,
 def backward(hidden: torch.Tensor, weight: torch.Tensor, labels: torch.Tensor,
              lse: torch.Tensor, grad_output: Optional[torch.Tensor] = None,
              grad_scale: float = 1.0, num_valid: Optional[torch.Tensor] = None,
+             num_label_tokens: Optional[int] = None,
              ignore_index: int = -100, softcap: float = 0.0, reduction: str = "sum",
              workspace: Optional[torch.Tensor] = None,
              d_hidden: Optional[torch.Tensor] = None, d_weight: Optional[torch.Tensor] = None,
@@ -132,7 +150,8 @@ def backward(hidden: torch.Tensor, weight: torch.Tensor, labels: torch.Tensor,
     added into the given d_hidden / d_weight instead of overwriting them (e.g.
     over the micro-batches of one optimizer step).  compute_d_weight=False
     (a frozen LM head) or compute_d_hidden=False skips that gradient's GEMM
-    and returns None in its place."""
+    and returns None in its place.  num_label_tokens as for forward: the
+    gradient of the normalised 'sum' loss."""
     h2, w, y = _prep(hidden, weight, labels)
     N, H = h2.shape
     V = w.shape[0]
@@ -174,11 +193,12 @@ def backward(hidden: torch.Tensor, weight: torch.Tensor, labels: torch.Tensor,
     if num_valid is not None:
         num_valid = num_valid.reshape(()).to(device=dev, dtype=torch.int64).contiguous()
     lse = lse.contiguous()
-    st = _lib().flce_backward(_ptr(h2), _ptr(w), _ptr(y), _ptr(lse), N, H, V, int(ignore_index),
-                              float(softcap), _REDUCTIONS[reduction], _DTYPES[h2.dtype],
-                              _ptr(grad_output), float(grad_scale), _ptr(num_valid),
-                              _ptr(d_hidden), _ptr(d_weight), flags, _ptr(workspace),
-                              workspace.numel(), _stream(dev))
+    st = _lib().flce_backward_ex(_ptr(h2), _ptr(w), _ptr(y), _ptr(lse), N, H, V,
+                                 int(ignore_index), float(softcap), _REDUCTIONS[reduction],
+                                 _DTYPES[h2.dtype], _ptr(grad_output), float(grad_scale),
+                                 _count(num_label_tokens), _ptr(num_valid), _ptr(d_hidden),
+                                 _ptr(d_weight), flags, _ptr(workspace), workspace.numel(),
+                                 _stream(dev))
     _native.check(st, "flce_backward")
     if check_status:
         _native.check(status(workspace), "flce_backward (device status)")
@@ -188,42 +208,47 @@ def backward(hidden: torch.Tensor, weight: torch.Tensor, labels: torch.Tensor,
 class _FlceFunction(torch.autograd.Function):
     @staticmethod
     def forward(ctx, hidden, weight, labels, ignore_index, softcap, reduction, grad_scale,
-                loss_scale):
+                loss_scale, num_label_tokens):
         out = forward(hidden, weight, labels, ignore_index, softcap, reduction,
-                      loss_scale=loss_scale)
+                      loss_scale=loss_scale, num_label_tokens=num_label_tokens)
         ctx.save_for_backward(hidden, weight, labels, out.lse)
-        # the returned loss is scaled by loss_scale, so is its gradient
-        ctx.cfg = (ignore_index, softcap, reduction, grad_scale * loss_scale, hidden.shape)
+        # the returned loss is scaled by loss_scale (and normalised by the count,
+        # in the library), so is its gradient
+        ctx.cfg = (ignore_index, softcap, reduction, grad_scale * loss_scale, num_label_tokens,
+                   hidden.shape)
         ctx.mark_non_differentiable(out.num_tokens)
         return out.loss, out.num_tokens
 
     @staticmethod
     def backward(ctx, grad_loss, _grad_ntok):
         hidden, weight, labels, lse = ctx.saved_tensors
-        ignore_index, softcap, reduction, grad_scale, hshape = ctx.cfg
+        ignore_index, softcap, reduction, grad_scale, num_label_tokens, hshape = ctx.cfg
         # gradients in the parameters' own dtype (bf16 rounded once from fp32),
         # and only those autograd asks for (a frozen LM head skips dWeight)
         need_dh, need_dw = ctx.needs_input_grad[0], ctx.needs_input_grad[1]
         if not (need_dh or need_dw):
-            return (None,) * 8
+            return (None,) * 9
         dh = (torch.empty(hshape, dtype=hidden.dtype, device=hidden.device)
               .view(-1, hshape[-1]) if need_dh else None)
         dw = torch.empty(weight.shape, dtype=weight.dtype, device=weight.device) \
             if need_dw else None
         backward(hidden, weight, labels, lse, grad_output=grad_loss, grad_scale=grad_scale,
-                 ignore_index=ignore_index, softcap=softcap, reduction=reduction,
-                 d_hidden=dh, d_weight=dw, compute_d_hidden=need_dh, compute_d_weight=need_dw)
-        return (dh.view(hshape) if need_dh else None), dw, None, None, None, None, None, None
+                 num_label_tokens=num_label_tokens, ignore_index=ignore_index, softcap=softcap,
+                 reduction=reduction, d_hidden=dh, d_weight=dw, compute_d_hidden=need_dh,
+                 compute_d_weight=need_dw)
+        return ((dh.view(hshape) if need_dh else None), dw) + (None,) * 7
 
 
 def fused_linear_cross_entropy(hidden, weight, labels, ignore_index: int = -100,
                                softcap: float = 0.0, reduction: str = "sum",
-                               grad_scale: float = 1.0, loss_scale: float = 1.0):
+                               grad_scale: float = 1.0, loss_scale: float = 1.0,
+                               num_label_tokens: Optional[int] = None):
     """Differentiable (loss, num_tokens); gradients flow to hidden and weight.
-    The loss is multiplied by loss_scale (and so is its gradient); grad_scale
-    scales the gradient alone (a micro-batch's token weighting)."""
+    The loss is multiplied by loss_scale and, for 'sum' with num_label_tokens,
+    normalised by that global count (so is its gradient); grad_scale scales the
+    gradient alone (a micro-batch's token weighting)."""
     return _FlceFunction.apply(hidden, weight, labels, ignore_index, softcap, reduction,
-                               grad_scale, loss_scale)
+                               grad_scale, loss_scale, num_label_tokens)
 
 
 class FusedLinearCrossEntropy(torch.nn.Module):
@@ -246,19 +271,17 @@ class FusedLinearCrossEntropy(torch.nn.Module):
                 grad_reduce_group=None, *, grad_scale: float = 1.0) -> torch.Tensor:
         """Loss of hidden_states [..., H] against labels [...] with lm_weight [V, H].
 
-        num_label_tokens: the global number of non-padding target tokens; a 'sum'
-        loss is divided by max(num_label_tokens, 1) (in the library's fp64 loss
-        sum) and so is its gradient.  Ignored for 'mean'.
+        num_label_tokens: the global number of non-padding target tokens; the
+        library divides a 'sum' loss by max(num_label_tokens, 1) (in its fp64
+        loss sum) and its gradient with it.  Ignored for 'mean'.
         grad_reduce_group: only None (one GPU, a regular lm_weight tensor).
         grad_scale: scales the gradient alone (micro-batch token weighting)."""
         if grad_reduce_group is not None:
             raise NotImplementedError("a sharded lm_weight (grad_reduce_group) is not "
                                       "supported: this loss runs on one GPU")
-        loss_scale = 1.0
-        if num_label_tokens is not None and self.reduction == "sum":
-            loss_scale = 1.0 / max(int(num_label_tokens), 1)
         loss, ntok = fused_linear_cross_entropy(hidden_states, lm_weight, labels,
                                                 self.ignore_index, self.logit_softcapping,
-                                                self.reduction, grad_scale, loss_scale)
+                                                self.reduction, grad_scale,
+                                                num_label_tokens=num_label_tokens)
         self.num_tokens = ntok
         return loss

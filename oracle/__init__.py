@@ -9,6 +9,6 @@ invariants, a pure-Python brute force and torch's CPU cross-entropy; see the
 module docstring of `oracle.flce_ref` for the definitions it follows.
 """
 from .flce_ref import (  # noqa: F401
-    MEAN, SUM, backward, capped_logits, d_hidden_rows, d_weight_rows, dlogits,
-    forward, grad_factor, label_logits, lse_rows, row_logsumexp,
+    MEAN, SUM, backward, capped_logits, d_hidden_rows, d_hidden_rows_sliced, d_weight_rows,
+    dlogits, forward, grad_factor, label_logits, lse_rows, lse_rows_sliced, row_logsumexp,
 )

@@ -236,3 +236,47 @@ def d_weight_rows(hidden: np.ndarray, weight: np.ndarray, labels: np.ndarray,
     G[labels == ignore_index] = 0.0
     G *= g
     return G.T @ h
+
+
+# ---------------------------------------------------------------------------
+# The same definitions with the sums over the vocabulary split into slices, for
+# a weight too large to hold on the host in float64 at once.  A logsumexp over
+# disjoint column sets combines as lse = log(sum_k exp(lse_k)), and dHidden is a
+# sum over vocabulary rows, so slicing changes only the order of the float64
+# additions.
+# ---------------------------------------------------------------------------
+
+def lse_rows_sliced(hidden: np.ndarray, weight: np.ndarray, rows: Sequence[int],
+                    softcap: float = 0.0, vocab_slice: int = 65536) -> np.ndarray:
+    """logsumexp of the selected rows, taken over vocabulary slices and combined."""
+    V = weight.shape[0]
+    parts = [lse_rows(hidden, weight[a:a + vocab_slice], rows, softcap)
+             for a in range(0, V, vocab_slice)]
+    return np.logaddexp.reduce(np.stack(parts), axis=0)
+
+
+def d_hidden_rows_sliced(hidden: np.ndarray, weight: np.ndarray, labels: np.ndarray,
+                         rows: Sequence[int], lse: np.ndarray, g: float,
+                         ignore_index: int = -100, softcap: float = 0.0,
+                         vocab_slice: int = 65536) -> np.ndarray:
+    """dHidden of the selected rows from their logsumexp `lse` (one value per
+    selected row), summed over vocabulary slices."""
+    rows = np.asarray(rows, dtype=np.int64)
+    labels = np.asarray(labels, dtype=np.int64)
+    y = labels[rows]
+    valid = y != ignore_index
+    lse = np.asarray(lse, dtype=np.float64)
+    h = _f64(hidden[rows])
+    V = weight.shape[0]
+    out = np.zeros((len(rows), hidden.shape[1]), dtype=np.float64)
+    for a in range(0, V, vocab_slice):
+        Wsl = _f64(weight[a:a + vocab_slice])
+        z, L = capped_logits(h, Wsl, softcap)
+        G = np.exp(L - lse[:, None])
+        here = np.nonzero(valid & (y >= a) & (y < a + Wsl.shape[0]))[0]
+        G[here, y[here] - a] -= 1.0
+        if softcap > 0:
+            G *= 1.0 - np.tanh(z / softcap) ** 2
+        G[~valid] = 0.0
+        out += G @ Wsl
+    return g * out

@@ -12,13 +12,11 @@ Tolerances come from the contract of this FLCE build:
                                   wide margin while still catching any
                                   dropped tile or wrong column (>= 1e-2).
 """
-import contextlib
-import os
-
 import numpy as np
 import torch
 
 import flce_inputs as fi
+from lm_head_linear_tmem_b200 import _native
 
 LOSS_RTOL = 1e-5
 GRAD_RL2 = 2e-3
@@ -58,21 +56,8 @@ def small_inputs(N, H, V, seed, n_ign, w_std=0.05):
     return fi.make_inputs(w, keep_raw=True)
 
 
-@contextlib.contextmanager
 def chunks(tokens: int, vocab: int):
     """Run the backward with tokens x vocab chunks instead of the default
     8192 x 16384, so that small problems span several chunks along both
-    reduced dimensions (FLCE_CHUNK_TOKENS / FLCE_CHUNK_VOCAB, read by the
-    library at every call)."""
-    keys = ("FLCE_CHUNK_TOKENS", "FLCE_CHUNK_VOCAB")
-    old = {k: os.environ.get(k) for k in keys}
-    os.environ["FLCE_CHUNK_TOKENS"] = str(tokens)
-    os.environ["FLCE_CHUNK_VOCAB"] = str(vocab)
-    try:
-        yield
-    finally:
-        for k, v in old.items():
-            if v is None:
-                os.environ.pop(k, None)
-            else:
-                os.environ[k] = v
+    reduced dimensions (library options FLCE_OPT_CHUNK_TOKENS / _VOCAB)."""
+    return _native.options(chunk_tokens=tokens, chunk_vocab=vocab)

@@ -117,6 +117,59 @@ def test_argument_errors_are_synchronous(lib):
                                    FAKE, FAKE, FAKE, FAKE, wsb, None) == ARG
 
 
+def test_options_host_side(lib):
+    """Options are set and read through the ABI (no environment variable reaches
+    the library); out-of-range values and unknown options are refused and leave
+    the option unchanged; the workspace size follows the chunk options."""
+    v = ctypes.c_int64()
+    defaults = {"cta_group": 2, "bwd_compact": 1, "bwd_fuse": 1, "mn3d": 1,
+                "chunk_tokens": 8192, "chunk_vocab": 16384, "wait_timeout_ms": 1000,
+                "grad_tile_n": 512, "dz_tile_n": 256, "fwd_tile_n": 256}
+    assert set(defaults) == set(_native.OPTIONS)
+    for name, dflt in defaults.items():
+        assert _native.get_option(name) == dflt, name
+    ARG = 1
+    for name, bad in (("cta_group", 3), ("cta_group", 0), ("bwd_compact", 2),
+                      ("chunk_tokens", 100), ("chunk_vocab", 1 << 21),
+                      ("wait_timeout_ms", 5), ("grad_tile_n", 384), ("dz_tile_n", 128),
+                      ("fwd_tile_n", 1024)):
+        assert lib.flce_set_option(_native.OPTIONS[name], bad) == ARG, (name, bad)
+        assert _native.get_option(name) == defaults[name]
+    assert lib.flce_set_option(-1, 0) == ARG and lib.flce_set_option(99, 0) == ARG
+    assert lib.flce_get_option(99, ctypes.byref(v)) == ARG
+    assert lib.flce_get_option(0, None) == ARG
+    big = lib.flce_workspace_bytes(16384, 4096, 131072, 0)
+    with _native.options(chunk_tokens=1024, chunk_vocab=2048, grad_tile_n=256):
+        assert _native.get_option("chunk_tokens") == 1024
+        assert _native.get_option("grad_tile_n") == 256
+        small = lib.flce_workspace_bytes(16384, 4096, 131072, 0)
+        assert small < big  # the dZ block is 1024 x 2048 bf16 instead of 8192 x 16384
+    assert _native.get_option("chunk_tokens") == 8192
+    assert _native.get_option("grad_tile_n") == 512
+    assert lib.flce_workspace_bytes(16384, 4096, 131072, 0) == big
+    # a chunk size that is not a multiple of 256 is rounded up
+    with _native.options(chunk_vocab=512):
+        ws512 = lib.flce_workspace_bytes(8192, 64, 5000, 0)
+    with _native.options(chunk_vocab=300):
+        assert _native.get_option("chunk_vocab") == 300
+        assert lib.flce_workspace_bytes(8192, 64, 5000, 0) == ws512
+
+
+def test_label_token_count_entry_points_host_side(lib):
+    """flce_forward_ex2 / flce_backward_ex check their arguments like the calls they
+    extend (the count itself is any int64: negative means none)."""
+    ARG = 1
+    wsb = lib.flce_workspace_bytes(64, 64, 512, 0)
+    assert lib.flce_forward_ex2(FAKE, FAKE, FAKE, 64, 64, 512, -100, 0.0, 5, 0, 1.0, 10,
+                                FAKE, FAKE, FAKE, FAKE, wsb, None) == ARG
+    assert lib.flce_forward_ex2(FAKE, FAKE, FAKE, 64, 64, 512, -100, 0.0, 0, 0, float("nan"),
+                                10, FAKE, FAKE, FAKE, FAKE, wsb, None) == ARG
+    assert lib.flce_backward_ex(FAKE, FAKE, FAKE, FAKE, 64, 64, 512, -100, 0.0, 0, 0, None,
+                                float("inf"), 10, None, FAKE, FAKE, 0, FAKE, wsb, None) == ARG
+    assert lib.flce_backward_ex(FAKE, FAKE, FAKE, FAKE, 64, 64, 512, -100, 0.0, 0, 0, None,
+                                1.0, 10, None, None, None, 0, FAKE, wsb, None) == ARG
+
+
 def test_profile_api_host_side(lib):
     ms = ctypes.c_double()
     n = ctypes.c_int64()

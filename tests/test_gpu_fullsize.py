@@ -4,8 +4,9 @@ benchmark times.
 The V=32000 problem is compared in full against the float64 oracle.  For the
 larger ones the oracle's full-size values (every row's logsumexp and label
 logit, the loss, the counts) were written by tests/golden/make_oracle_fullsize.py,
-which calls only the oracle; dHidden and dWeight are compared on seeded
-samples of rows that the oracle computes one by one.
+which calls only the oracle; dHidden is compared on 4096 seeded token rows and
+dWeight on 4096 seeded vocabulary rows (the most frequent labels and both ends
+among them), which the oracle computes one by one on the host cores.
 """
 import os
 
@@ -20,6 +21,8 @@ from tests import _gpu as G
 
 pytestmark = pytest.mark.gpu
 IGN = fi.IGNORE_INDEX
+SAMPLE_ROWS = 4096   # dHidden token rows compared at full size
+SAMPLE_VOCAB = 4096  # dWeight vocabulary rows compared at full size
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 
@@ -82,10 +85,10 @@ def _check_sampled(inp, gold, lse_gpu, dh, dw, g, seed):
     ign = inp.labels == IGN
     assert np.all(dh[ign] == 0.0)
     assert np.all(np.isfinite(dh))
-    rows = sample_rows(inp.labels, 256, seed)
+    rows = sample_rows(inp.labels, SAMPLE_ROWS, seed)
     ref_dh = oracle.d_hidden_rows(H64, W64, inp.labels, rows, g, IGN, w.softcap)
     assert G.rel_l2(dh[rows], ref_dh) <= G.GRAD_RL2
-    vrows = sample_vocab(inp.labels, w.V, 512, seed)
+    vrows = sample_vocab(inp.labels, w.V, SAMPLE_VOCAB, seed)
     ref_dw = oracle.d_weight_rows(H64, W64, inp.labels, vrows, gold["lse"], g, IGN, w.softcap)
     got_dw = dw[vrows]
     assert np.all(np.isfinite(got_dw))
@@ -160,9 +163,10 @@ def test_flat_offsets_beyond_int32():
     """V*H > 2^31: the top vocabulary rows of W and dWeight lie past the int32
     range of flat element offsets.  Half of the valid rows take labels there, so
     the dZ label entries, the dHidden W-row gathers and the dWeight label-term
-    sums all touch those rows; lse and the loss are checked on every row and
-    dWeight on the top rows (plus a sample), against the oracle on vocabulary
-    slices combined by the logsumexp identity lse = log(sum_k exp(lse_k))."""
+    sums all touch those rows; lse and the loss are checked on every row,
+    dWeight on the top rows (plus a sample) and dHidden on rows labelled in the
+    top rows (plus ignored and low-label rows), against the oracle evaluated
+    over vocabulary slices."""
     N, H, V = 256, 4096, (1 << 19) + 512  # V*H = 2^31 + 2^21 elements
     w = fi.custom_workload(N, H, V, seed=41, w_std=0.02, ignore_count=16)
     inp = fi.make_inputs(w)
@@ -185,9 +189,7 @@ def test_flat_offsets_beyond_int32():
     loss = f.loss.item()
     del dw, dh, W
     torch.cuda.empty_cache()
-    parts = [oracle.lse_rows(inp.hidden, inp.weight[a:a + 65536], np.arange(N))
-             for a in range(0, V, 65536)]
-    lse_ref = np.logaddexp.reduce(np.stack(parts), axis=0)
+    lse_ref = oracle.lse_rows_sliced(inp.hidden, inp.weight, np.arange(N), vocab_slice=65536)
     assert np.max(np.abs(lse_gpu - lse_ref)) <= G.LSE_ATOL
     ll = oracle.label_logits(inp.hidden, inp.weight, y, IGN)
     G.check_loss(loss, float(np.sum((lse_ref - ll)[y != IGN])))
@@ -196,3 +198,13 @@ def test_flat_offsets_beyond_int32():
     assert G.rel_l2(dw_rows, ref_dw) <= G.GRAD_RL2
     assert G.rel_l2(dw_rows[64:], ref_dw[64:]) <= G.GRAD_RL2  # the rows past 2^31
     assert np.all(dh_np[y == IGN] == 0.0) and np.all(np.isfinite(dh_np))
+    # dHidden rows whose label entry gathers a W row past 2^31 elements, plus a few
+    # rows with low labels and ignored rows
+    top_rows = np.nonzero(y >= V - 512)[0]
+    other = np.nonzero((y < V - 512) & (y != IGN))[0][:16]
+    ign_rows = np.nonzero(y == IGN)[0][:4]
+    rows = np.sort(np.concatenate([top_rows, other, ign_rows]))
+    ref_dh = oracle.d_hidden_rows_sliced(inp.hidden, inp.weight, y, rows, lse_ref[rows], 1.0,
+                                         IGN, vocab_slice=65536)
+    assert G.rel_l2(dh_np[rows], ref_dh) <= G.GRAD_RL2
+    assert G.rel_l2(dh_np[top_rows], ref_dh[np.isin(rows, top_rows)]) <= G.GRAD_RL2

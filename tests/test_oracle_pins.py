@@ -263,6 +263,35 @@ def test_row_sampled_forms_match_full():
                            b["d_weight"][vr], rtol=1e-12, atol=1e-16)
 
 
+def test_vocab_sliced_forms_match_brute_force_and_full():
+    """The vocabulary-sliced lse and dHidden (for weights too large for host
+    memory in float64) against the pure-Python brute force with finite
+    differences, and against the unsliced forms, with slices that do not divide V
+    and labels in every slice."""
+    h, w, y = small_problem(N=4, H=3, V=8, seed=31, w_std=0.8, n_ign=1)
+    for s in (0.0, 1.5):
+        rows = [0, 1, 2, 3]
+        lse = oracle.lse_rows_sliced(h, w, rows, s, vocab_slice=3)
+        for i in rows:
+            L = [s * math.tanh(float(np.dot(h[i], wv)) / s) if s > 0 else float(np.dot(h[i], wv))
+                 for wv in w]
+            assert abs(lse[i] - math.log(sum(math.exp(v) for v in L))) < 1e-12
+        dh_bf, _ = _brute.finite_diff(h.tolist(), w.tolist(), y.tolist(), IGN, s, "sum")
+        got = oracle.d_hidden_rows_sliced(h, w, y, rows, lse, 1.0, IGN, s, vocab_slice=3)
+        assert np.allclose(got, np.array(dh_bf), atol=1e-7, rtol=1e-6)
+    h, w, y = small_problem(N=30, H=6, V=50, seed=32, n_ign=6)
+    for s in (0.0, 2.5):
+        rows = [0, 4, 9, 29]
+        ref_lse = oracle.lse_rows(h, w, rows, s)
+        for k in (1, 7, 50, 64):
+            lse = oracle.lse_rows_sliced(h, w, rows, s, vocab_slice=k)
+            assert np.allclose(lse, ref_lse, rtol=1e-14, atol=0)
+            assert np.allclose(oracle.d_hidden_rows_sliced(h, w, y, rows, lse, 0.3, IGN, s,
+                                                           vocab_slice=k),
+                               oracle.d_hidden_rows(h, w, y, rows, 0.3, IGN, s),
+                               rtol=1e-12, atol=1e-16)
+
+
 # --------------------------------------------------------------------------
 # values printed by the pages
 # --------------------------------------------------------------------------
