@@ -114,7 +114,12 @@ typedef enum flce_option {
                                    with FLCE_OPT_CTA_GROUP = 1 tiles are 256 wide) */
   FLCE_OPT_DZ_TILE_N = 8,       /* [256] columns of a backward dZ tile: 256 or 512 (as above) */
   FLCE_OPT_FWD_TILE_N = 9,      /* [256] columns of a forward tile: 256 or 512 (as above) */
-  FLCE_OPT_COUNT_ = 10          /* number of options (not an option) */
+  FLCE_OPT_FWD_GROUP_M = 10,    /* [16] row tiles per raster group of the forward GEMM (1 .. 64): the
+                                   group's hidden rows stay in L2 while the weight streams past */
+  FLCE_OPT_DZ_GROUP_M = 11,     /* [16] the same for the backward dZ GEMM */
+  FLCE_OPT_GRAD_GROUP_M = 12,   /* [8] the same for the dHidden / dWeight GEMMs */
+  FLCE_OPT_FWD_DYNAMIC = 13,    /* [1] forward tiles are handed out by an atomic counter; 0: round-robin */
+  FLCE_OPT_COUNT_ = 14          /* number of options (not an option) */
 } flce_option;
 
 /* Set option `option` to `value`.  FLCE_ERR_ARG for an unknown option or a

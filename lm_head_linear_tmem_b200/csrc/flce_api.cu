@@ -219,11 +219,16 @@ constexpr OptSpec kOptSpec[kNumOpts] = {
     {512, 256, 512},           // FLCE_OPT_GRAD_TILE_N
     {256, 256, 512},           // FLCE_OPT_DZ_TILE_N
     {256, 256, 512},           // FLCE_OPT_FWD_TILE_N
+    {kGroupM, 1, 64},          // FLCE_OPT_FWD_GROUP_M
+    {kGroupM, 1, 64},          // FLCE_OPT_DZ_GROUP_M
+    {kGroupMGrad, 1, 64},      // FLCE_OPT_GRAD_GROUP_M
+    {1, 0, 1},                 // FLCE_OPT_FWD_DYNAMIC
 };
 std::atomic<int64_t> g_opt[kNumOpts] = {
     {kOptSpec[0].dflt}, {kOptSpec[1].dflt}, {kOptSpec[2].dflt}, {kOptSpec[3].dflt},
     {kOptSpec[4].dflt}, {kOptSpec[5].dflt}, {kOptSpec[6].dflt}, {kOptSpec[7].dflt},
-    {kOptSpec[8].dflt}, {kOptSpec[9].dflt}};
+    {kOptSpec[8].dflt}, {kOptSpec[9].dflt}, {kOptSpec[10].dflt}, {kOptSpec[11].dflt},
+    {kOptSpec[12].dflt}, {kOptSpec[13].dflt}};
 
 struct Opts {
   int cta_group;          // 2: CTA pairs with 256-row tiles; 1: single CTAs, 128-row tiles
@@ -236,6 +241,8 @@ struct Opts {
   int grad_bn;            // columns of a dHidden / dWeight tile (512 needs CTA pairs)
   int dz_bn;              // columns of a dZ tile
   int fwd_bn;             // columns of a forward tile
+  int fwd_group, dz_group, grad_group;  // row tiles per raster group (L2 reuse)
+  bool fwd_dynamic;       // forward tiles handed out by an atomic counter (else round-robin)
 };
 
 Opts opts() {
@@ -250,6 +257,10 @@ Opts opts() {
   o.grad_bn = (o.cta_group == 2) ? static_cast<int>(g_opt[FLCE_OPT_GRAD_TILE_N].load()) : 256;
   o.dz_bn = (o.cta_group == 2) ? static_cast<int>(g_opt[FLCE_OPT_DZ_TILE_N].load()) : 256;
   o.fwd_bn = (o.cta_group == 2) ? static_cast<int>(g_opt[FLCE_OPT_FWD_TILE_N].load()) : 256;
+  o.fwd_group = static_cast<int>(g_opt[FLCE_OPT_FWD_GROUP_M].load());
+  o.dz_group = static_cast<int>(g_opt[FLCE_OPT_DZ_GROUP_M].load());
+  o.grad_group = static_cast<int>(g_opt[FLCE_OPT_GRAD_GROUP_M].load());
+  o.fwd_dynamic = g_opt[FLCE_OPT_FWD_DYNAMIC].load() != 0;
   return o;
 }
 
@@ -354,7 +365,10 @@ GradScratch grad_scratch(const Opts& o, int64_t N, int64_t H, int64_t V, bool bf
   return g;
 }
 
+// Workspace header (256 B; its first 16 bytes are zeroed by every forward):
+// status word at 0, the forward's tile counter at 4, n_valid at 8.
 unsigned int* ws_status(void* ws) { return reinterpret_cast<unsigned int*>(ws); }
+int* ws_fwd_counter(void* ws) { return reinterpret_cast<int*>(static_cast<char*>(ws) + 4); }
 long long* ws_nvalid(void* ws) {
   return reinterpret_cast<long long*>(reinterpret_cast<char*>(ws) + 8);
 }
@@ -505,11 +519,14 @@ flce_status forward_bf16(DevInfo* d, const Opts& o, const void* hidden, const vo
 
   GemmArgs g{};
   g.k_blocks = static_cast<int>((H + BK - 1) / BK);
-  g.group_m = kGroupM;
+  g.group_m = o.fwd_group;
   g.a_off = 0;
   g.b_off = 0;
   g.status = ws_status(ws);
   g.timeout_ns = o.timeout_ns;
+  // dynamic hand-out keeps the pairs in step across the raster's waves, so the
+  // weight panels a wave shares are still in L2 when its last pair reads them
+  g.tile_counter = o.fwd_dynamic ? ws_fwd_counter(ws) : nullptr;
 
   cudaError_t e;
   const GemmProblem prob{&ta, &tb, &ta, N, V, g};
@@ -732,7 +749,7 @@ flce_status backward_bf16(DevInfo* d, const Opts& o, const void* hidden, const v
       // 1) dZ = f(hidden[t0:] . W[v0:]^T) -> bf16 block
       GemmArgs gz{};
       gz.k_blocks = k_blocks_h;
-      gz.group_m = kGroupM;
+      gz.group_m = o.dz_group;
       gz.a_off = static_cast<int>(t0);
       gz.b_off = static_cast<int>(v0);
       gz.status = ws_status(ws);
@@ -762,7 +779,7 @@ flce_status backward_bf16(DevInfo* d, const Opts& o, const void* hidden, const v
       // 2) dHidden[t0:t0+rows] (+)= dZ . W[v0:v0+cols]
       GemmArgs gh{};
       gh.k_blocks = (cols + BK - 1) / BK;
-      gh.group_m = kGroupMGrad;
+      gh.group_m = o.grad_group;
       gh.a_off = 0;
       gh.b_off = static_cast<int>(v0);
       gh.status = ws_status(ws);
@@ -785,7 +802,7 @@ flce_status backward_bf16(DevInfo* d, const Opts& o, const void* hidden, const v
       // 3) dWeight[v0:v0+cols] (+)= dZ^T . hidden[t0:t0+rows]
       GemmArgs gw{};
       gw.k_blocks = (rows + BK - 1) / BK;
-      gw.group_m = kGroupMGrad;
+      gw.group_m = o.grad_group;
       gw.a_off = 0;
       gw.b_off = static_cast<int>(t0);
       gw.status = ws_status(ws);
