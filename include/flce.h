@@ -104,7 +104,7 @@ typedef enum flce_option {
                                    (and then also skips the exact fp32 label-term correction) */
   FLCE_OPT_BWD_FUSE = 2,        /* [1] dHidden and dWeight GEMMs of a backward chunk share one launch; 0: two */
   FLCE_OPT_MN3D = 3,            /* [1] MN-major operands load through 3-D chunk views; 0: 2-D views */
-  FLCE_OPT_CHUNK_TOKENS = 4,    /* [8192] token rows of a backward chunk (256 .. 2^20, rounded up to 256) */
+  FLCE_OPT_CHUNK_TOKENS = 4,    /* [16384] token rows of a backward chunk (256 .. 2^20, rounded up to 256) */
   FLCE_OPT_CHUNK_VOCAB = 5,     /* [16384] vocab columns of a backward chunk (256 .. 2^20, rounded up to 256);
                                    the dZ block of the workspace is chunk_tokens x chunk_vocab bf16, so
                                    flce_workspace_bytes must be called with the same chunk options as the
@@ -113,13 +113,15 @@ typedef enum flce_option {
   FLCE_OPT_GRAD_TILE_N = 7,     /* [512] columns of a dHidden / dWeight tile: 512 or 256 (512 needs CTA pairs;
                                    with FLCE_OPT_CTA_GROUP = 1 tiles are 256 wide) */
   FLCE_OPT_DZ_TILE_N = 8,       /* [256] columns of a backward dZ tile: 256 or 512 (as above) */
-  FLCE_OPT_FWD_TILE_N = 9,      /* [256] columns of a forward tile: 256 or 512 (as above) */
+  FLCE_OPT_FWD_TILE_N = 9,      /* [512] columns of a forward tile: 512 or 256 (as above) */
   FLCE_OPT_FWD_GROUP_M = 10,    /* [16] row tiles per raster group of the forward GEMM (1 .. 64): the
                                    group's hidden rows stay in L2 while the weight streams past */
   FLCE_OPT_DZ_GROUP_M = 11,     /* [16] the same for the backward dZ GEMM */
   FLCE_OPT_GRAD_GROUP_M = 12,   /* [8] the same for the dHidden / dWeight GEMMs */
   FLCE_OPT_FWD_DYNAMIC = 13,    /* [1] forward tiles are handed out by an atomic counter; 0: round-robin */
-  FLCE_OPT_COUNT_ = 14          /* number of options (not an option) */
+  FLCE_OPT_DZ_BUFFERS = 14,     /* [1] backward dZ blocks in the workspace: 1, or 2 (each chunk's dZ GEMM
+                                   then runs beside the previous chunk's gradient GEMMs) */
+  FLCE_OPT_COUNT_ = 15          /* number of options (not an option) */
 } flce_option;
 
 /* Set option `option` to `value`.  FLCE_ERR_ARG for an unknown option or a

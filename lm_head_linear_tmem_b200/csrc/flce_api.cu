@@ -31,11 +31,14 @@
 namespace flce {
 namespace {
 
-// Backward chunk: kChunkTokens x kChunkVocab (dZ block 256 MiB bf16).  Longer
-// tiles along the reduced dimensions (K = 16384 for dHidden, 8192 for
-// dWeight) and fewer fp32 read-add-write passes over dHidden and dWeight
-// measured faster than an L2-sized 4096 x 8192 block.
-constexpr int kChunkTokens = 8192;
+// Backward chunk: kChunkTokens x kChunkVocab (dZ block 512 MiB bf16, 1/8 of
+// the [16384, 131072] dZ of the bench problem).  Longer tiles along the
+// reduced dimensions (K = 16384 for dHidden, up to 16384 for dWeight), fewer
+// launches and fewer fp32 read-add-write passes over dHidden and dWeight: one
+// token chunk writes dWeight once.  Measured at the power cap (interleaved
+// A/B): 16384 x 16384 chunks 0.5% faster than 8192 x 16384, which was 6%
+// faster than an L2-sized 4096 x 8192 block.
+constexpr int kChunkTokens = 16384;
 constexpr int kChunkVocab = 16384;
 constexpr int kGroupM = 16;     // forward and dZ
 constexpr int kGroupMGrad = 8;  // dHidden and dWeight: their long-K panels (8 MiB at the bench
@@ -218,17 +221,18 @@ constexpr OptSpec kOptSpec[kNumOpts] = {
     {1000, 10, 60000},         // FLCE_OPT_WAIT_TIMEOUT_MS
     {512, 256, 512},           // FLCE_OPT_GRAD_TILE_N
     {256, 256, 512},           // FLCE_OPT_DZ_TILE_N
-    {256, 256, 512},           // FLCE_OPT_FWD_TILE_N
+    {512, 256, 512},           // FLCE_OPT_FWD_TILE_N
     {kGroupM, 1, 64},          // FLCE_OPT_FWD_GROUP_M
     {kGroupM, 1, 64},          // FLCE_OPT_DZ_GROUP_M
     {kGroupMGrad, 1, 64},      // FLCE_OPT_GRAD_GROUP_M
     {1, 0, 1},                 // FLCE_OPT_FWD_DYNAMIC
+    {1, 1, 2},                 // FLCE_OPT_DZ_BUFFERS
 };
 std::atomic<int64_t> g_opt[kNumOpts] = {
     {kOptSpec[0].dflt}, {kOptSpec[1].dflt}, {kOptSpec[2].dflt}, {kOptSpec[3].dflt},
     {kOptSpec[4].dflt}, {kOptSpec[5].dflt}, {kOptSpec[6].dflt}, {kOptSpec[7].dflt},
     {kOptSpec[8].dflt}, {kOptSpec[9].dflt}, {kOptSpec[10].dflt}, {kOptSpec[11].dflt},
-    {kOptSpec[12].dflt}, {kOptSpec[13].dflt}};
+    {kOptSpec[12].dflt}, {kOptSpec[13].dflt}, {kOptSpec[14].dflt}};
 
 struct Opts {
   int cta_group;          // 2: CTA pairs with 256-row tiles; 1: single CTAs, 128-row tiles
@@ -243,6 +247,8 @@ struct Opts {
   int fwd_bn;             // columns of a forward tile
   int fwd_group, dz_group, grad_group;  // row tiles per raster group (L2 reuse)
   bool fwd_dynamic;       // forward tiles handed out by an atomic counter (else round-robin)
+  int dz_buffers;         // backward dZ blocks: 2 lets a chunk's dZ run beside the previous
+                          // chunk's gradient GEMMs
 };
 
 Opts opts() {
@@ -261,6 +267,7 @@ Opts opts() {
   o.dz_group = static_cast<int>(g_opt[FLCE_OPT_DZ_GROUP_M].load());
   o.grad_group = static_cast<int>(g_opt[FLCE_OPT_GRAD_GROUP_M].load());
   o.fwd_dynamic = g_opt[FLCE_OPT_FWD_DYNAMIC].load() != 0;
+  o.dz_buffers = static_cast<int>(g_opt[FLCE_OPT_DZ_BUFFERS].load());
   return o;
 }
 
@@ -284,12 +291,15 @@ Chunking chunking(const Opts& o, int64_t N, int64_t V) {
   return c;
 }
 
-// Backward GEMM launches of one call (at most three per chunk), each with its
-// own dynamic tile counter in the workspace.
-int64_t bwd_launches(const Opts& o, int64_t N, int64_t V) {
+int64_t bwd_chunks(const Opts& o, int64_t N, int64_t V) {
   const Chunking c = chunking(o, N, V);
-  return 3 * ((N + c.tc - 1) / c.tc) * ((V + c.vc - 1) / c.vc);
+  return ((N + c.tc - 1) / c.tc) * ((V + c.vc - 1) / c.vc);
 }
+
+// Backward counters of one call, zeroed at its start: a dynamic tile counter
+// for each GEMM launch (at most three per chunk), then one per chunk that the
+// CTAs of its gradient launches count themselves out on.
+int64_t bwd_counters(const Opts& o, int64_t N, int64_t V) { return 4 * bwd_chunks(o, N, V); }
 
 // Backward workspace: header | tile counters | row compaction (permutation,
 // compact labels and lse, per-block counts, valid count) | label sort (two
@@ -298,7 +308,7 @@ int64_t bwd_launches(const Opts& o, int64_t N, int64_t V) {
 // reuse once the GEMMs are done.
 struct BwdLayout {
   size_t counters, perm, labels_c, lse_c, block_valid, n_valid_c, keys0, keys1, vals0, vals1,
-      hist, resid, hidden_c, gblock, part, end;
+      hist, resid, hidden_c, gblock, gblock_bytes, part, end;
 };
 
 BwdLayout bwd_layout(const Opts& o, int64_t N, int64_t H, int64_t V) {
@@ -307,7 +317,7 @@ BwdLayout bwd_layout(const Opts& o, int64_t N, int64_t H, int64_t V) {
   const size_t nblk = static_cast<size_t>((N + kCompactThreads - 1) / kCompactThreads);
   size_t off = kHeaderBytes;
   L.counters = off;
-  off = align_up(off + 4 * static_cast<size_t>(bwd_launches(o, N, V)), 256);
+  off = align_up(off + 4 * static_cast<size_t>(bwd_counters(o, N, V)), 256);
   L.perm = off;
   off = align_up(off + 4 * static_cast<size_t>(N), 256);
   L.labels_c = off;
@@ -327,9 +337,10 @@ BwdLayout bwd_layout(const Opts& o, int64_t N, int64_t H, int64_t V) {
   L.hidden_c = off;
   off = align_up(off + 2 * static_cast<size_t>(N) * static_cast<size_t>(H), 1024);
   L.gblock = off;
+  L.gblock_bytes = align_up(static_cast<size_t>(c.tc) * c.vc * 2 + 1024, 1024);
   L.part = off;
   const size_t nseg = static_cast<size_t>((N + kFixSeg - 1) / kFixSeg);
-  off += std::max(static_cast<size_t>(c.tc) * c.vc * 2 + 1024,
+  off += std::max(L.gblock_bytes * static_cast<size_t>(o.dz_buffers),
                   nseg * 2 * static_cast<size_t>(H) * 4);
   L.end = off;
   return L;
@@ -434,7 +445,7 @@ struct GemmProblem {
 template <class Epi, int kCG, int kBN, bool kAMn0, bool kBMn0, bool kAMn1, bool kBMn1>
 cudaError_t run_gemm_cg(DevInfo* d, int kind, const GemmProblem& p0,
                         const typename Epi::Params& ep0, const GemmProblem* p1,
-                        const typename Epi::Params& ep1, cudaStream_t st) {
+                        const typename Epi::Params& ep1, cudaStream_t st, int* ctas_out) {
   using Cfg = TileCfg<kCG, kBN>;
   auto k = tc_gemm_kernel<Epi, kCG, kBN, kAMn0, kBMn0, kAMn1, kBMn1>;
   cudaError_t e = set_smem_attr(k, Cfg::kSmemBytes);
@@ -452,6 +463,7 @@ cudaError_t run_gemm_cg(DevInfo* d, int kind, const GemmProblem& p0,
   const GemmProblem& q1 = p1 ? *p1 : p0;
   const int tiles = g0.m_tiles * g0.n_tiles + g1.m_tiles * g1.n_tiles;
   const int units = std::max(1, std::min(tiles, d->sms / kCG));
+  if (ctas_out != nullptr) *ctas_out = units * kCG;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(units * kCG, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -483,16 +495,21 @@ cudaError_t run_gemm_cg(DevInfo* d, int kind, const GemmProblem& p0,
 }
 
 // The launch in the CTA group of `o` with tiles of `bn` columns (512 only
-// with CTA pairs; opts() guarantees it).
+// with CTA pairs; opts() guarantees it).  *ctas_out (if given) receives the
+// number of CTAs launched.
 template <class Epi, bool kAMn0, bool kBMn0, bool kAMn1 = false, bool kBMn1 = false>
 cudaError_t run_gemm(DevInfo* d, const Opts& o, int bn, int kind, const GemmProblem& p0,
                      const typename Epi::Params& ep0, const GemmProblem* p1,
-                     const typename Epi::Params& ep1, cudaStream_t st) {
+                     const typename Epi::Params& ep1, cudaStream_t st,
+                     int* ctas_out = nullptr) {
   if (o.cta_group == 1)
-    return run_gemm_cg<Epi, 1, 256, kAMn0, kBMn0, kAMn1, kBMn1>(d, kind, p0, ep0, p1, ep1, st);
+    return run_gemm_cg<Epi, 1, 256, kAMn0, kBMn0, kAMn1, kBMn1>(d, kind, p0, ep0, p1, ep1, st,
+                                                                ctas_out);
   if (bn == 512)
-    return run_gemm_cg<Epi, 2, 512, kAMn0, kBMn0, kAMn1, kBMn1>(d, kind, p0, ep0, p1, ep1, st);
-  return run_gemm_cg<Epi, 2, 256, kAMn0, kBMn0, kAMn1, kBMn1>(d, kind, p0, ep0, p1, ep1, st);
+    return run_gemm_cg<Epi, 2, 512, kAMn0, kBMn0, kAMn1, kBMn1>(d, kind, p0, ep0, p1, ep1, st,
+                                                                ctas_out);
+  return run_gemm_cg<Epi, 2, 256, kAMn0, kBMn0, kAMn1, kBMn1>(d, kind, p0, ep0, p1, ep1, st,
+                                                              ctas_out);
 }
 
 // Rows of B (K-major) one CTA stages per bank and K-block.
@@ -618,11 +635,13 @@ flce_status backward_bf16(DevInfo* d, const Opts& o, const void* hidden, const v
   const Chunking ck = chunking(o, N, V);
   const BwdLayout BL = bwd_layout(o, N, H, V);
   char* w = static_cast<char*>(ws);
-  void* gbuf = w + BL.gblock;
   int* counters = reinterpret_cast<int*>(w + BL.counters);
   int next_counter = 0;
+  const int nchunks = static_cast<int>(bwd_chunks(o, N, V));
+  int* done = counters + 3 * nchunks;  // per chunk: CTAs of its gradient launches that finished
+  std::vector<int> readers(nchunks, 0);  // per chunk: CTAs of its gradient launches
   {
-    const cudaError_t e = cudaMemsetAsync(counters, 0, 4 * bwd_launches(o, N, V), st);
+    const cudaError_t e = cudaMemsetAsync(counters, 0, 4 * bwd_counters(o, N, V), st);
     if (e != cudaSuccess) return cuda_fail(e);
   }
 
@@ -728,11 +747,14 @@ flce_status backward_bf16(DevInfo* d, const Opts& o, const void* hidden, const v
   const unsigned long long tmo = o.timeout_ns;
   const int mean = reduction == FLCE_MEAN;
 
+  int ci = 0;  // chunk index
   for (int64_t t0 = 0; t0 < N; t0 += ck.tc) {
     const int rows = static_cast<int>(std::min<int64_t>(ck.tc, N - t0));
-    for (int64_t v0 = 0; v0 < V; v0 += ck.vc) {
+    for (int64_t v0 = 0; v0 < V; v0 += ck.vc, ++ci) {
       const int cols = static_cast<int>(std::min<int64_t>(ck.vc, V - v0));
-      // dZ block [rows, cols] bf16, row stride ck.vc elements.
+      // dZ block [rows, cols] bf16, row stride ck.vc elements (one of dz_buffers
+      // blocks, used by chunks in turn)
+      void* gbuf = w + BL.gblock + static_cast<size_t>(ci % o.dz_buffers) * BL.gblock_bytes;
       CUtensorMap t_g_store, t_g_k, t_g_mn;
       if (!make_map(&t_g_store, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, gbuf, cols, rows,
                     static_cast<uint64_t>(ck.vc) * 2, 64, 32) ||
@@ -759,9 +781,24 @@ flce_status backward_bf16(DevInfo* d, const Opts& o, const void* hidden, const v
       gz.rows_base = static_cast<int>(t0);
       gz.rows_host = rows;
       gz.rows_dim = kRowsM;
-      // dZ overwrites the block the previous chunk's dHidden/dWeight GEMMs read:
-      // its main loop may start early, its first store waits for them
-      gz.dep_wait = (t0 > 0 || v0 > 0) ? kDepBeforeStores : kDepNone;
+      if (ci == 0) {
+        gz.dep_wait = kDepNone;
+      } else if (o.dz_buffers == 1) {
+        // dZ overwrites the block the previous chunk's dHidden/dWeight GEMMs
+        // read: its main loop may start early, its first store waits for them
+        gz.dep_wait = kDepBeforeStores;
+      } else {
+        // two blocks: dZ runs beside the previous chunk's gradient GEMMs (in
+        // their last wave), stores once the chunk before that, which read this
+        // block, has counted all its CTAs out, and completes only after the
+        // previous launch, so the next gradient launch, which waits for this
+        // one, also follows the previous one
+        gz.dep_wait = kDepBeforeExit;
+        if (ci >= 2) {
+          gz.wait_counter = done + (ci - 2);
+          gz.wait_target = readers[ci - 2];
+        }
+      }
       cudaError_t e;
       const GemmProblem pz{&t_hid_k, &t_w_k, &t_g_store, rows, cols, gz};
       if (softcap > 0.f) {
@@ -791,6 +828,7 @@ flce_status backward_bf16(DevInfo* d, const Opts& o, const void* hidden, const v
       gh.rows_dim = kRowsM;
       gh.dep_wait = kDepBeforeLoads;  // reads the dZ block written just before
       gh.b_mn3d = h3d ? 1 : 0;
+      if (o.dz_buffers > 1) gh.done_counter = done + ci;
       // the last vocab chunk's dHidden epilogue also adds the exact label term
       const bool last_v = v0 + ck.vc >= V;
       StoreEpi::Params eh{static_cast<int>(t0), (v0 > 0 || acc_dh) ? 1 : 0, static_cast<int>(H),
@@ -816,6 +854,7 @@ flce_status backward_bf16(DevInfo* d, const Opts& o, const void* hidden, const v
       gw.dep_wait = kDepBeforeLoads;
       gw.a_mn3d = mn3d ? 1 : 0;
       gw.b_mn3d = h3d ? 1 : 0;
+      if (o.dz_buffers > 1) gw.done_counter = done + ci;
       StoreEpi::Params ew{static_cast<int>(v0), (t0 > 0 || acc_dw) ? 1 : 0, static_cast<int>(H),
                           static_cast<int>(V), grad_output, grad_scale, n_valid, mean,
                           nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0};
@@ -823,14 +862,21 @@ flce_status backward_bf16(DevInfo* d, const Opts& o, const void* hidden, const v
       const GemmProblem ph{&t_g_k, &t_w_mn, &t_dh, rows, H, gh};
       const GemmProblem pw{&t_g_mn, &t_hid_mn, &t_dw, cols, H, gw};
       const int gbn = o.grad_bn;
+      int ctas = 0;
       if (want_dh && want_dw && o.fuse) {
         // 2) + 3) in one launch: the dWeight tiles fill the dHidden grid's last wave
-        e = run_gemm<StoreEpi, false, true, true, true>(d, o, gbn, kBwdDhDw, ph, eh, &pw, ew, st);
+        e = run_gemm<StoreEpi, false, true, true, true>(d, o, gbn, kBwdDhDw, ph, eh, &pw, ew, st,
+                                                        &ctas);
+        readers[ci] += ctas;
       } else {
-        if (want_dh)
-          e = run_gemm<StoreEpi, false, true>(d, o, gbn, kBwdDhDw, ph, eh, nullptr, eh, st);
-        if (want_dw && e == cudaSuccess)
-          e = run_gemm<StoreEpi, true, true>(d, o, gbn, kBwdDhDw, pw, ew, nullptr, ew, st);
+        if (want_dh) {
+          e = run_gemm<StoreEpi, false, true>(d, o, gbn, kBwdDhDw, ph, eh, nullptr, eh, st, &ctas);
+          readers[ci] += ctas;
+        }
+        if (want_dw && e == cudaSuccess) {
+          e = run_gemm<StoreEpi, true, true>(d, o, gbn, kBwdDhDw, pw, ew, nullptr, ew, st, &ctas);
+          readers[ci] += ctas;
+        }
       }
       if (e != cudaSuccess) return cuda_fail(e);
     }

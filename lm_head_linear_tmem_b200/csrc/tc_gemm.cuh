@@ -96,7 +96,15 @@ struct GemmArgs {
                       // nullptr: static round-robin over the CTAs (or CTA pairs)
   int dep_wait;       // what waits for the previous kernel on the stream (launched
                       // as a programmatic dependent): kDepNone, kDepBeforeLoads
-                      // (operands it produced), kDepBeforeStores (an output it reads)
+                      // (operands it produced), kDepBeforeStores (an output it reads),
+                      // kDepBeforeExit (only completion order: the grid does not
+                      // complete before the previous one)
+  // Before its first store the epilogue waits (bounded) until *wait_counter
+  // reaches wait_target: the CTAs of an earlier launch that read what this
+  // launch overwrites count themselves out there.  Null: no wait.
+  const int* wait_counter;
+  int wait_target;
+  int* done_counter;  // every CTA adds 1 here when it has finished (null: none)
   // Token rows bounded on the device: when rows_valid is set, only the first
   // clamp(*rows_valid - rows_base, 0, rows_host) token rows of this launch are
   // worked on.  rows_dim says which GEMM dimension they are (kRowsM, kRowsK);
@@ -121,6 +129,7 @@ constexpr int kRowsK = 2;
 constexpr int kDepNone = 0;
 constexpr int kDepBeforeLoads = 1;
 constexpr int kDepBeforeStores = 2;
+constexpr int kDepBeforeExit = 3;
 
 __device__ __forceinline__ void tile_coords(int tile, const GemmArgs& g, int& mb, int& nb) {
   const int per_group = g.group_m * g.n_tiles;
@@ -864,16 +873,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------- epilogue warps (they may read what the previous kernel
-    // wrote, so they wait for it in either mode)
-    if (g0.dep_wait != kDepNone) griddep_wait();
+    // wrote, so they wait for it in either of the first two modes)
+    if (g0.dep_wait == kDepBeforeLoads || g0.dep_wait == kDepBeforeStores) griddep_wait();
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     uint8_t* stg = smem + kStages * Cfg::kStageBytes + (warp - 2) * kStagingPerWarp;
     int it = 0;
     int nstore = 0;  // TMA stores issued by this warp (selects the staging buffer)
     bool ok = true;
+    if (g0.wait_counter != nullptr) {
+      // the launch that last read what this one overwrites has finished
+      bool w = true;
+      if (lane == 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_acquire_gpu(g0.wait_counter) < g0.wait_target) {
+          if (*abort_flag || globaltimer_ns() - t0 > g0.timeout_ns) {
+            w = false;
+            break;
+          }
+          __nanosleep(256);
+        }
+        fence_proxy_async_global();
+      }
+      ok = __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
+    }
     int rslot = 0;
     uint32_t rph = 0;
-    for (;; ++it) {
+    for (; ok; ++it) {
       int tile;
       ok = ring_take(rslot, rph, true, tile);
       if (++rslot == kRing) {
@@ -920,6 +945,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     else
       tmem_dealloc_pair(tmem_base, kTmemCols);
   }
+  // every operand load of this CTA has been consumed and every store waited for
+  if (g0.done_counter != nullptr && threadIdx.x == 0) red_release_gpu_add(g0.done_counter, 1);
+  if (g0.dep_wait == kDepBeforeExit && threadIdx.x == 0) griddep_wait();
 }
 
 }  // namespace flce

@@ -57,8 +57,8 @@ def test_workspace_bytes(lib):
     big = ws(16384, 4096, 131072, 0)
     # forward partials: 512 vocab tiles x 16384 rows x (m, s) fp32 = 64 MiB;
     # backward: compact hidden 16384 x 4096 bf16 = 128 MiB + dZ block
-    # 8192 x 16384 bf16 = 256 MiB + row-compaction, label-sort and residual arrays
-    assert 384 * 2 ** 20 <= big < 386 * 2 ** 20
+    # 16384 x 16384 bf16 = 512 MiB + row-compaction, label-sort and residual arrays
+    assert 640 * 2 ** 20 <= big < 642 * 2 ** 20
     assert ws(0, 64, 512, 0) > 0
     assert ws(64, 64, 512, 1) > 0
     ex = lib.flce_workspace_bytes_ex
@@ -123,9 +123,10 @@ def test_options_host_side(lib):
     the option unchanged; the workspace size follows the chunk options."""
     v = ctypes.c_int64()
     defaults = {"cta_group": 2, "bwd_compact": 1, "bwd_fuse": 1, "mn3d": 1,
-                "chunk_tokens": 8192, "chunk_vocab": 16384, "wait_timeout_ms": 1000,
-                "grad_tile_n": 512, "dz_tile_n": 256, "fwd_tile_n": 256, "fwd_group_m": 16,
-                "dz_group_m": 16, "grad_group_m": 8, "fwd_dynamic": 1}
+                "chunk_tokens": 16384, "chunk_vocab": 16384, "wait_timeout_ms": 1000,
+                "grad_tile_n": 512, "dz_tile_n": 256, "fwd_tile_n": 512, "fwd_group_m": 16,
+                "dz_group_m": 16, "grad_group_m": 8, "fwd_dynamic": 1,
+                "dz_buffers": 1}
     assert set(defaults) == set(_native.OPTIONS)
     for name, dflt in defaults.items():
         assert _native.get_option(name) == dflt, name
@@ -144,8 +145,8 @@ def test_options_host_side(lib):
         assert _native.get_option("chunk_tokens") == 1024
         assert _native.get_option("grad_tile_n") == 256
         small = lib.flce_workspace_bytes(16384, 4096, 131072, 0)
-        assert small < big  # the dZ block is 1024 x 2048 bf16 instead of 8192 x 16384
-    assert _native.get_option("chunk_tokens") == 8192
+        assert small < big  # the dZ block is 1024 x 2048 bf16 instead of 16384 x 16384
+    assert _native.get_option("chunk_tokens") == 16384
     assert _native.get_option("grad_tile_n") == 512
     assert lib.flce_workspace_bytes(16384, 4096, 131072, 0) == big
     # a chunk size that is not a multiple of 256 is rounded up

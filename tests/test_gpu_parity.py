@@ -192,13 +192,17 @@ def test_module_autograd_and_num_tokens_contract():
         assert G.rel_l2(w.grad.float().cpu().numpy(), bf16_round(rb["d_weight"])) <= G.GRAD_RL2
 
 
-def test_repeated_calls_are_deterministic():
+@pytest.mark.parametrize("buffers", [1, 2])
+def test_repeated_calls_are_deterministic(buffers):
+    """Every sum has a fixed order: repeated calls agree bit for bit, and one or two
+    dZ blocks (which only change which launches overlap) give the same bits."""
     inp = G.small_inputs(N=4200, H=128, V=8500, seed=14, n_ign=100)
     args = (G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
             G.labels_tensor(inp.labels), 0.0, "sum")
     with G.chunks(*SMALL_CHUNKS):
         a = run(*args)
-        b = run(*args)
+        with _native.options(dz_buffers=buffers):
+            b = run(*args)
     assert a["loss"] == b["loss"]
     assert np.array_equal(a["lse"], b["lse"])
     assert np.array_equal(a["dh"], b["dh"]) and np.array_equal(a["dw"], b["dw"])
@@ -372,15 +376,20 @@ def test_degenerate_shapes(N, H, V, dtype):
 
 
 @pytest.mark.parametrize("switch", ["cta_group=1", "bwd_fuse=0", "bwd_compact=0", "mn3d=0",
-                                    "grad_tile_n=256", "dz_tile_n=512", "fwd_tile_n=512"])
+                                    "grad_tile_n=256", "dz_tile_n=512", "fwd_tile_n=256",
+                                    "fwd_dynamic=0", "dz_buffers=2", "dz_buffers=2,bwd_fuse=0",
+                                    "dz_buffers=2,cta_group=1", "fwd_group_m=3,dz_group_m=2,"
+                                    "grad_group_m=1"])
 def test_alternative_paths(switch):
     """Each schedule option of the library selects another correct path: single-CTA
     128 x 256 tiles, separate dHidden and dWeight launches, no row compaction (and
     so no exact label term), 2-D views for MN-major operands, 256-column gradient
-    tiles, 512-column dZ and forward tiles."""
-    key, val = switch.split("=")
+    and forward tiles, 512-column dZ tiles, round-robin forward tiles, two dZ
+    blocks (9 chunks here, so a dZ launch waits on the gradient launches two
+    chunks back before it overwrites their block), other raster groups."""
+    opts = {kv.split("=")[0]: int(kv.split("=")[1]) for kv in switch.split(",")}
     inp = G.small_inputs(N=2100, H=192, V=4500, seed=26, n_ign=300, w_std=0.1)
-    with _native.options(**{key: int(val)}), G.chunks(*SMALL_CHUNKS):
+    with _native.options(**opts), G.chunks(*SMALL_CHUNKS):
         got = run(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
                   G.labels_tensor(inp.labels), 2.0, "mean", grad_scale=0.7)
     compare(got, inp.hidden, inp.weight, inp.labels, 2.0, "mean", grad_scale=0.7)

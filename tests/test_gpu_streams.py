@@ -11,6 +11,7 @@ import torch
 
 import flce_inputs as fi
 import lm_head_linear_tmem_b200 as flce
+from lm_head_linear_tmem_b200 import _native
 from tests import _gpu as G
 
 pytestmark = pytest.mark.gpu
@@ -30,13 +31,15 @@ def _eager(h, W, y, softcap):
     return f.loss.clone(), f.lse.clone(), dh, dw
 
 
-@pytest.mark.parametrize("softcap", [0.0, 3.0])
-def test_graph_capture_replays_identically(softcap):
+@pytest.mark.parametrize("softcap,buffers", [(0.0, 1), (3.0, 1), (3.0, 2)])
+def test_graph_capture_replays_identically(softcap, buffers):
     h, W, y = _problem(30)
     h2, _, y2 = _problem(31)
     N, H = h.shape
     V = W.shape[0]
-    with G.chunks(1024, 2048):  # several chunks, so the capture holds the whole schedule
+    # several chunks, so the capture holds the whole schedule (with two dZ blocks,
+    # the chunks' dZ and gradient launches overlap inside the graph)
+    with G.chunks(1024, 2048), _native.options(dz_buffers=buffers):
         ref1 = _eager(h, W, y, softcap)
         ref2 = _eager(h2, W, y2, softcap)
         hs, ys = h.clone(), y.clone()  # the graph's static inputs
