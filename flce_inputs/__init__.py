@@ -92,13 +92,15 @@ WORKLOADS: Dict[str, Workload] = {
         description="N=16384 as 4 micro-batches of 4096, micro-batch 1 all ignored, "
                     "others 30% ignored, sum with token-weighted grad scale"),
     # A smaller problem whose backward launches have exactly the per-launch
-    # shapes of v131k_zipf (H=4096; 8192-token x 16384-vocab backward chunks),
-    # used for profiler captures that must stay small on the device.
-    "profile_8k": Workload(
-        name="profile_8k", N=8192, H=4096, V=32768, batch_shape=(1, 8192), w_std=0.02,
-        labels="zipf1.1", ignore_rule="count", ignore_count=409, softcap=0.0,
+    # shapes of v131k_zipf (N=16384, H=4096; 16384-token x 16384-vocab backward
+    # chunks) and whose forward is a quarter of its forward (V=32768), used for
+    # profiler captures that must stay small on the device (about 2 GB).
+    "profile_16k": Workload(
+        name="profile_16k", N=16384, H=4096, V=32768, batch_shape=(2, 8192), w_std=0.02,
+        labels="zipf1.1", ignore_rule="count", ignore_count=819, softcap=0.0,
         reduction="sum", seed=6,
-        description="N=8192 H=4096 V=32768, Zipf(1.1) labels, 5% ignored, sum (profiling size)"),
+        description="N=16384 H=4096 V=32768, Zipf(1.1) labels, 5% ignored, sum "
+                    "(profiling size)"),
 }
 
 # The order of the five problems as they are listed for this workload family.
