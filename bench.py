@@ -417,16 +417,19 @@ def run_own(args, rank, world, local_rank):
 
     peaks, peak_src = load_peaks()
     flops_step = w.flops_per_step
-    # Work the kernels execute: the forward covers every row; the backward GEMMs
-    # cover the non-ignored rows only (rows with ignore_index have exactly zero
-    # gradient and are compacted away) unless the bwd_compact option is off.
+    # Work the kernels execute: the forward and backward GEMMs cover the
+    # non-ignored rows only (rows with ignore_index take no part in the loss and
+    # have exactly zero gradient; they are compacted away) unless the
+    # fwd_compact / bwd_compact options are off.  The credited work counts every
+    # row: 8*N*H*V.
     n_valid = int((inp.labels != fi.IGNORE_INDEX).sum())
-    compact = _native.get_option("bwd_compact") != 0
-    n_bwd = n_valid if compact else N
-    executed_step = 2.0 * N * H * V + 6.0 * n_bwd * H * V
-    # the dominant kernel (largest device time) and its roofline
-    # FLOP per step of each kernel kind (summed over its launches)
-    credited = {"fwd_gemm_softmax_stats": 2.0 * N * H * V, "bwd_dz_gemm": 2.0 * n_bwd * H * V,
+    n_bwd = n_valid if _native.get_option("bwd_compact") != 0 else N
+    n_fwd = n_valid if _native.get_option("fwd_compact") != 0 else N
+    executed_step = 2.0 * n_fwd * H * V + 6.0 * n_bwd * H * V
+    # the dominant kernel (largest device time) and its roofline, from the FLOP
+    # each kernel kind executes per step (summed over its launches)
+    credited = {"fwd_gemm_softmax_stats": 2.0 * n_fwd * H * V,
+                "bwd_dz_gemm": 2.0 * n_bwd * H * V,
                 "bwd_dhidden_dweight_gemm": 4.0 * n_bwd * H * V}
     dom = max(kinds, key=lambda k: kinds[k]["ms_total"]) if kinds else None
     roofline = None
@@ -474,7 +477,7 @@ def run_own(args, rank, world, local_rank):
                             "executed_tflops": executed_step / (ms_step / 1e3) / 1e12,
                             "executed_frac_of_sustained":
                                 executed_step / (ms_step / 1e3) / 1e12 / sust,
-                            "backward_rows": n_bwd, "tokens": N,
+                            "forward_rows": n_fwd, "backward_rows": n_bwd, "tokens": N,
                             "peak_source": peak_src},
         "roofline": roofline,
         "gemm_roofline": gemm_roofline,

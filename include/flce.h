@@ -121,7 +121,9 @@ typedef enum flce_option {
   FLCE_OPT_FWD_DYNAMIC = 13,    /* [1] forward tiles are handed out by an atomic counter; 0: round-robin */
   FLCE_OPT_DZ_BUFFERS = 14,     /* [1] backward dZ blocks in the workspace: 1, or 2 (each chunk's dZ GEMM
                                    then runs beside the previous chunk's gradient GEMMs) */
-  FLCE_OPT_COUNT_ = 15          /* number of options (not an option) */
+  FLCE_OPT_FWD_COMPACT = 15,    /* [1] the bf16 forward compacts the rows that take part in the loss and
+                                   runs its GEMM on those alone; 0: on every row (same results) */
+  FLCE_OPT_COUNT_ = 16          /* number of options (not an option) */
 } flce_option;
 
 /* Set option `option` to `value`.  FLCE_ERR_ARG for an unknown option or a
@@ -144,7 +146,10 @@ size_t flce_workspace_bytes_ex(int64_t N, int64_t H, int64_t V, int32_t dtype, i
 /* Forward.
  *   loss        device float[1]   'sum' or 'mean' loss (float32)
  *   num_tokens  device int64[1]   n for 'sum', 0 for 'mean'
- *   lse         device float[N]   log-sum-exp of every row (ignored rows included);
+ *   lse         device float[N]   log-sum-exp of every row that takes part in the loss;
+ *                                 0 for a row whose label is ignore_index (or outside
+ *                                 [0, V)): neither the loss nor its gradient depends on
+ *                                 those rows, so their logits are not computed.
  *                                 flce_backward reads it.
  * ignore_index may be any int64; a row is ignored iff labels[i] == ignore_index.
  * softcap must be >= 0 (0 = off).  The async status word is cleared first. */

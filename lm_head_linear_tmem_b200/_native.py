@@ -34,7 +34,7 @@ OPTIONS = {
     "cta_group": 0, "bwd_compact": 1, "bwd_fuse": 2, "mn3d": 3, "chunk_tokens": 4,
     "chunk_vocab": 5, "wait_timeout_ms": 6, "grad_tile_n": 7, "dz_tile_n": 8, "fwd_tile_n": 9,
     "fwd_group_m": 10, "dz_group_m": 11, "grad_group_m": 12, "fwd_dynamic": 13,
-    "dz_buffers": 14,
+    "dz_buffers": 14, "fwd_compact": 15,
 }
 
 # Every symbol include/flce.h declares, with its ctypes signature.

@@ -179,11 +179,16 @@ bool make_map_mn3d(CUtensorMap* m, const void* base, uint64_t mn, uint64_t k_row
 // ---------------------------------------------------------------- workspace
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Forward workspace: header | softmax partials m, s [ceil(V/256), N] | label
+// logits [N] | per-block loss partials | and, when the rows are compacted
+// (bf16 path), the permutation, compact labels and lse, per-block counts, the
+// valid count and the compact hidden copy [N, H] bf16.
 struct FwdLayout {
   size_t part_m, part_s, label_logit, block_loss, block_cnt, end;
+  size_t perm, labels_c, lse_c, block_valid, n_valid_c, hidden_c, end_compact;
 };
 
-FwdLayout fwd_layout(int64_t N, int64_t V, bool bf16) {
+FwdLayout fwd_layout(int64_t N, int64_t V, bool bf16, int64_t H = 0) {
   FwdLayout L{};
   size_t off = kHeaderBytes;
   const size_t n_vt = bf16 ? static_cast<size_t>((V + BN - 1) / BN) : 0;
@@ -199,6 +204,20 @@ FwdLayout fwd_layout(int64_t N, int64_t V, bool bf16) {
   L.block_cnt = off;
   off = align_up(off + nblk * sizeof(long long), 256);
   L.end = off;
+  const size_t cblk = static_cast<size_t>((N + kCompactThreads - 1) / kCompactThreads);
+  L.perm = off;
+  off = align_up(off + 4 * static_cast<size_t>(N), 256);
+  L.labels_c = off;
+  off = align_up(off + 8 * static_cast<size_t>(N), 256);
+  L.lse_c = off;
+  off = align_up(off + 4 * static_cast<size_t>(N), 256);
+  L.block_valid = off;
+  off = align_up(off + 4 * cblk, 256);
+  L.n_valid_c = off;
+  off = align_up(off + 8, 1024);
+  L.hidden_c = off;
+  off = align_up(off + 2 * static_cast<size_t>(N) * static_cast<size_t>(H), 256);
+  L.end_compact = off;
   return L;
 }
 
@@ -227,12 +246,13 @@ constexpr OptSpec kOptSpec[kNumOpts] = {
     {kGroupMGrad, 1, 64},      // FLCE_OPT_GRAD_GROUP_M
     {1, 0, 1},                 // FLCE_OPT_FWD_DYNAMIC
     {1, 1, 2},                 // FLCE_OPT_DZ_BUFFERS
+    {1, 0, 1},                 // FLCE_OPT_FWD_COMPACT
 };
 std::atomic<int64_t> g_opt[kNumOpts] = {
     {kOptSpec[0].dflt}, {kOptSpec[1].dflt}, {kOptSpec[2].dflt}, {kOptSpec[3].dflt},
     {kOptSpec[4].dflt}, {kOptSpec[5].dflt}, {kOptSpec[6].dflt}, {kOptSpec[7].dflt},
     {kOptSpec[8].dflt}, {kOptSpec[9].dflt}, {kOptSpec[10].dflt}, {kOptSpec[11].dflt},
-    {kOptSpec[12].dflt}, {kOptSpec[13].dflt}, {kOptSpec[14].dflt}};
+    {kOptSpec[12].dflt}, {kOptSpec[13].dflt}, {kOptSpec[14].dflt}, {kOptSpec[15].dflt}};
 
 struct Opts {
   int cta_group;          // 2: CTA pairs with 256-row tiles; 1: single CTAs, 128-row tiles
@@ -249,6 +269,7 @@ struct Opts {
   bool fwd_dynamic;       // forward tiles handed out by an atomic counter (else round-robin)
   int dz_buffers;         // backward dZ blocks: 2 lets a chunk's dZ run beside the previous
                           // chunk's gradient GEMMs
+  bool fwd_compact;       // the bf16 forward leaves rows outside the loss out of its GEMM
 };
 
 Opts opts() {
@@ -268,6 +289,7 @@ Opts opts() {
   o.grad_group = static_cast<int>(g_opt[FLCE_OPT_GRAD_GROUP_M].load());
   o.fwd_dynamic = g_opt[FLCE_OPT_FWD_DYNAMIC].load() != 0;
   o.dz_buffers = static_cast<int>(g_opt[FLCE_OPT_DZ_BUFFERS].load());
+  o.fwd_compact = g_opt[FLCE_OPT_FWD_COMPACT].load() != 0;
   return o;
 }
 
@@ -352,7 +374,9 @@ size_t bwd_bytes(const Opts& o, int64_t N, int64_t H, int64_t V, bool bf16) {
 }
 
 size_t ws_bytes(const Opts& o, int64_t N, int64_t H, int64_t V, bool bf16) {
-  return align_up(std::max(fwd_layout(N, V, bf16).end, bwd_bytes(o, N, H, V, bf16)), 256);
+  const FwdLayout F = fwd_layout(N, V, bf16, H);
+  const size_t fwd = (bf16 && o.fwd_compact) ? F.end_compact : F.end;
+  return align_up(std::max(fwd, bwd_bytes(o, N, H, V, bf16)), 256);
 }
 
 // bf16 gradient outputs: fp32 scratch for dHidden and/or dWeight after the
@@ -516,21 +540,67 @@ cudaError_t run_gemm(DevInfo* d, const Opts& o, int bn, int kind, const GemmProb
 uint32_t b_box_rows(const Opts& o) { return static_cast<uint32_t>(BN / o.cta_group); }
 
 // ---------------------------------------------------------------- forward
+// `compact`: the rows outside the loss (ignore_index, or a label outside
+// [0, V)) are left out of the GEMM: the valid rows are compacted first (the
+// backward's stable compaction and hidden-row gather), the GEMM's token rows
+// are bounded by the device-side count, and the merge writes each lse back
+// through the permutation.  Either way such rows get lse 0.
 flce_status forward_bf16(DevInfo* d, const Opts& o, const void* hidden, const void* weight,
                          const int64_t* labels, int64_t N, int64_t H, int64_t V,
                          int64_t ignore_index, float softcap, int32_t reduction,
                          double loss_scale, double loss_div, float* loss, int64_t* num_tokens,
-                         float* lse, void* ws, cudaStream_t st) {
+                         float* lse, void* ws, cudaStream_t st, bool compact) {
   char* w = static_cast<char*>(ws);
-  const FwdLayout L = fwd_layout(N, V, true);
+  const FwdLayout L = fwd_layout(N, V, true, H);
   float* part_m = reinterpret_cast<float*>(w + L.part_m);
   float* part_s = reinterpret_cast<float*>(w + L.part_s);
   float* label_logit = reinterpret_cast<float*>(w + L.label_logit);
   double* block_loss = reinterpret_cast<double*>(w + L.block_loss);
   long long* block_cnt = reinterpret_cast<long long*>(w + L.block_cnt);
+  const int n = static_cast<int>(N);
+  cudaError_t e;
+
+  const void* hid = hidden;
+  const int64_t* lab = labels;
+  int* perm = nullptr;
+  long long* n_valid_c = nullptr;
+  float* lse_c = nullptr;
+  if (compact) {
+    perm = reinterpret_cast<int*>(w + L.perm);
+    int64_t* labels_c = reinterpret_cast<int64_t*>(w + L.labels_c);
+    lse_c = reinterpret_cast<float*>(w + L.lse_c);
+    int* block_valid = reinterpret_cast<int*>(w + L.block_valid);
+    n_valid_c = reinterpret_cast<long long*>(w + L.n_valid_c);
+    void* hidden_c = w + L.hidden_c;
+    const int cblk = (n + kCompactThreads - 1) / kCompactThreads;
+    e = launch(kHelper, st, [&] {
+      compact_count_kernel<<<cblk, kCompactThreads, 0, st>>>(labels, n, ignore_index, V,
+                                                             ws_status(ws), block_valid);
+    });
+    if (e == cudaSuccess)
+      e = launch(kHelper, st, [&] {
+        exclusive_scan_kernel<<<1, kCompactThreads, 0, st>>>(block_valid, cblk, n_valid_c);
+      });
+    if (e == cudaSuccess)
+      e = launch(kHelper, st, [&] {
+        compact_scatter_kernel<<<cblk, kCompactThreads, 0, st>>>(
+            labels, nullptr, n, ignore_index, block_valid, n_valid_c, perm, labels_c, nullptr, V,
+            nullptr, nullptr);
+      });
+    if (e == cudaSuccess)
+      e = launch(kHelper, st, [&] {
+        gather_rows_kernel<<<n, 256, 0, st>>>(static_cast<const uint4*>(hidden),
+                                              static_cast<int>(H / 8), n, perm, n_valid_c,
+                                              static_cast<uint4*>(hidden_c), nullptr,
+                                              static_cast<int>(H / 4), 0);
+      });
+    if (e != cudaSuccess) return cuda_fail(e);
+    hid = hidden_c;
+    lab = labels_c;
+  }
 
   CUtensorMap ta, tb;
-  if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hidden, H, N, H * 2, BK, BM) ||
+  if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hid, H, N, H * 2, BK, BM) ||
       !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, weight, H, V, H * 2, BK, b_box_rows(o)))
     return FLCE_ERR_CUDA;
 
@@ -544,33 +614,40 @@ flce_status forward_bf16(DevInfo* d, const Opts& o, const void* hidden, const vo
   // dynamic hand-out keeps the pairs in step across the raster's waves, so the
   // weight panels a wave shares are still in L2 when its last pair reads them
   g.tile_counter = o.fwd_dynamic ? ws_fwd_counter(ws) : nullptr;
+  if (compact) {  // only the valid (compacted) rows are worked on
+    g.rows_valid = n_valid_c;
+    g.rows_base = 0;
+    g.rows_host = n;
+    g.rows_dim = kRowsM;
+  }
 
-  cudaError_t e;
   const GemmProblem prob{&ta, &tb, &ta, N, V, g};
   if (softcap > 0.f) {
-    FwdStatsEpi<true>::Params ep{labels, static_cast<int>(N), static_cast<int>(V), softcap,
-                                 1.0f / softcap, part_m, part_s, label_logit};
+    FwdStatsEpi<true>::Params ep{lab, n, static_cast<int>(V), softcap, 1.0f / softcap, part_m,
+                                 part_s, label_logit};
     e = run_gemm<FwdStatsEpi<true>, false, false>(d, o, o.fwd_bn, kFwdGemm, prob, ep, nullptr,
                                                   ep, st);
   } else {
-    FwdStatsEpi<false>::Params ep{labels, static_cast<int>(N), static_cast<int>(V), 0.f, 0.f,
-                                  part_m, part_s, label_logit};
+    FwdStatsEpi<false>::Params ep{lab, n, static_cast<int>(V), 0.f, 0.f, part_m, part_s,
+                                  label_logit};
     e = run_gemm<FwdStatsEpi<false>, false, false>(d, o, o.fwd_bn, kFwdGemm, prob, ep, nullptr,
                                                    ep, st);
   }
   if (e != cudaSuccess) return cuda_fail(e);
 
-  const int n = static_cast<int>(N);
   const int n_vt = static_cast<int>((V + BN - 1) / BN);  // (m, s) partials per row
   e = launch(kFwdMerge, st, [&] {
     fwd_merge_kernel<<<(n + kMergeRows - 1) / kMergeRows, dim3(kMergeRows, kMergeSplit), 0, st>>>(
-        part_m, part_s, n_vt, n, lse);
+        part_m, part_s, n_vt, n, lse, labels, ignore_index, V, perm, n_valid_c, lse_c);
   });
   if (e != cudaSuccess) return cuda_fail(e);
+  // per-row losses in compact order when compacted (the rows past the valid
+  // ones carry ignore_index and add nothing)
   const int nblk = (n + kLossThreads - 1) / kLossThreads;
   e = launch(kFwdMerge, st, [&] {
-    row_loss_kernel<<<nblk, kLossThreads, 0, st>>>(lse, label_logit, labels, n, ignore_index, V,
-                                                   block_loss, block_cnt, ws_status(ws));
+    row_loss_kernel<<<nblk, kLossThreads, 0, st>>>(compact ? lse_c : lse, label_logit, lab, n,
+                                                   ignore_index, V, block_loss, block_cnt,
+                                                   ws_status(ws));
   });
   if (e != cudaSuccess) return cuda_fail(e);
   e = launch(kFwdMerge, st, [&] {
@@ -603,7 +680,7 @@ flce_status forward_fp32(DevInfo* d, const void* hidden, const void* weight,
   e = launch(kSimt, st, [&] {
     simt_fwd_kernel<<<n, kSimtThreads, h * sizeof(float), st>>>(
         static_cast<const float*>(hidden), static_cast<const float*>(weight), labels, n, h, v,
-        softcap, lse, label_logit);
+        softcap, ignore_index, lse, label_logit);
   });
   if (e != cudaSuccess) return cuda_fail(e);
   const int nblk = (n + kLossThreads - 1) / kLossThreads;
@@ -1004,7 +1081,7 @@ flce_status flce_forward_ex2(const void* hidden, const void* weight, const int64
   const double div = label_token_divisor(reduction, num_label_tokens);
   if (dtype == FLCE_BF16)
     return forward_bf16(d, o, hidden, weight, labels, N, H, V, ignore_index, softcap, reduction,
-                        loss_scale, div, loss, num_tokens, lse, workspace, st);
+                        loss_scale, div, loss, num_tokens, lse, workspace, st, o.fwd_compact);
   return forward_fp32(d, hidden, weight, labels, N, H, V, ignore_index, softcap, reduction,
                       loss_scale, div, loss, num_tokens, lse, workspace, st);
 }
@@ -1284,7 +1361,7 @@ extern "C" flce_status flce_forward_noalloc(const void* hidden, const void* weig
   } else {
     s = (dtype == FLCE_BF16)
             ? forward_bf16(d, opts(), hidden, weight, labels, N, H, V, ignore_index, softcap,
-                           reduction, 1.0, 1.0, loss, num_tokens, lse, ws, st)
+                           reduction, 1.0, 1.0, loss, num_tokens, lse, ws, st, false)
             : forward_fp32(d, hidden, weight, labels, N, H, V, ignore_index, softcap, reduction,
                            1.0, 1.0, loss, num_tokens, lse, ws, st);
     if (s != FLCE_OK) return s;

@@ -27,29 +27,54 @@ __device__ __forceinline__ void merge_ms(float& M, float& S, float m, float s) {
   }
 }
 
-// lse[row] = ln 2 * (M + log2 S) over all vocab tiles of the row.
-// Block (32 rows, 8 splits); grid ceil(N / 32).
+// lse = ln 2 * (M + log2 S) over all vocab tiles of a row, for the rows that
+// take part in the loss; a row whose label is ignore_index (or outside
+// [0, V)) gets lse 0 and no merge.  Block (32 rows, 8 splits); grid ceil(N/32).
+//   perm == nullptr: the partials are indexed by row; a row's label decides.
+//   perm != nullptr: the forward ran on compacted rows: partial column j is
+//     compact row j, the original row perm[j]; the first *n_valid compact rows
+//     take part.  lse_c[j] receives the value as well (compact order).
 __global__ void __launch_bounds__(kMergeRows * kMergeSplit)
     fwd_merge_kernel(const float* __restrict__ part_m, const float* __restrict__ part_s,
-                     int n_vt, int N, float* __restrict__ lse) {
+                     int n_vt, int N, float* __restrict__ lse, const int64_t* __restrict__ labels,
+                     int64_t ignore_index, int64_t V, const int* __restrict__ perm,
+                     const long long* __restrict__ n_valid, float* __restrict__ lse_c) {
   __shared__ float sm[kMergeSplit][kMergeRows];
   __shared__ float ss[kMergeSplit][kMergeRows];
   const int tx = threadIdx.x, ty = threadIdx.y;
-  const int row = blockIdx.x * kMergeRows + tx;
+  const int j = blockIdx.x * kMergeRows + tx;
+  bool live = j < N;
+  if (live) {
+    if (perm != nullptr) {
+      live = j < *n_valid;
+    } else {
+      const int64_t y = labels[j];
+      live = (y != ignore_index) && y >= 0 && y < V;
+    }
+  }
   float M = -CUDART_INF_F, S = 0.f;
-  if (row < N) {
+  if (live) {
     for (int vt = ty; vt < n_vt; vt += kMergeSplit) {
-      const size_t idx = static_cast<size_t>(vt) * N + row;
+      const size_t idx = static_cast<size_t>(vt) * N + j;
       merge_ms(M, S, part_m[idx], part_s[idx]);
     }
   }
   sm[ty][tx] = M;
   ss[ty][tx] = S;
   __syncthreads();
-  if (ty == 0 && row < N) {
-    float Mt = -CUDART_INF_F, St = 0.f;
-    for (int k = 0; k < kMergeSplit; ++k) merge_ms(Mt, St, sm[k][tx], ss[k][tx]);
-    lse[row] = (Mt + log2f(St)) * kLn2;
+  if (ty == 0 && j < N) {
+    float v = 0.f;
+    if (live) {
+      float Mt = -CUDART_INF_F, St = 0.f;
+      for (int k = 0; k < kMergeSplit; ++k) merge_ms(Mt, St, sm[k][tx], ss[k][tx]);
+      v = (Mt + log2f(St)) * kLn2;
+    }
+    if (perm != nullptr) {
+      lse[perm[j]] = v;
+      lse_c[j] = v;
+    } else {
+      lse[j] = v;
+    }
   }
 }
 
@@ -267,7 +292,8 @@ __global__ void __launch_bounds__(kCompactThreads)
 }
 
 // perm[j], and the compact labels and lse of every compact row: valid rows keep
-// theirs; ignored rows get ignore_index and lse 0.
+// theirs; ignored rows get ignore_index and lse 0.  lse / lse_c and the sort
+// keys may be null (the forward's compaction has no lse yet and no sort).
 __global__ void __launch_bounds__(kCompactThreads)
     compact_scatter_kernel(const int64_t* __restrict__ labels, const float* __restrict__ lse,
                            int N, int64_t ignore_index, const int* __restrict__ block_offset,
@@ -290,8 +316,8 @@ __global__ void __launch_bounds__(kCompactThreads)
     const int j = v ? rank_v : static_cast<int>(*n_valid) + (i - rank_v);
     perm[j] = i;
     labels_c[j] = v ? y : ignore_index;
-    lse_c[j] = v ? lse[i] : 0.f;
-    if (v) {  // the key is the label (in [0, V) for every compacted row)
+    if (lse_c != nullptr) lse_c[j] = v ? lse[i] : 0.f;
+    if (v && sort_keys != nullptr) {  // the key is the label (in [0, V) for every compacted row)
       sort_keys[j] = static_cast<uint32_t>(y);
       sort_vals[j] = i;
     }
@@ -553,11 +579,19 @@ __device__ __forceinline__ float capped(float z, float softcap) {
 __global__ void __launch_bounds__(kSimtThreads)
     simt_fwd_kernel(const float* __restrict__ hidden, const float* __restrict__ weight,
                     const int64_t* __restrict__ labels, int N, int H, int V, float softcap,
-                    float* __restrict__ lse, float* __restrict__ label_logit) {
+                    int64_t ignore_index, float* __restrict__ lse,
+                    float* __restrict__ label_logit) {
   extern __shared__ float sh[];
   __shared__ float red_m[kSimtThreads], red_s[kSimtThreads];
   const int row = blockIdx.x;
   const int t = threadIdx.x;
+  {  // a row outside the loss gets lse 0 and no work
+    const int64_t y0 = labels[row];
+    if (y0 == ignore_index || y0 < 0 || y0 >= V) {
+      if (t == 0) lse[row] = 0.f;
+      return;
+    }
+  }
   for (int k = t; k < H; k += kSimtThreads) sh[k] = hidden[static_cast<size_t>(row) * H + k];
   __syncthreads();
   const int64_t y = labels[row];

@@ -43,6 +43,19 @@ def rel_l2(got: np.ndarray, ref: np.ndarray) -> float:
     return num / den
 
 
+def check_lse(got: np.ndarray, ref: np.ndarray, labels: np.ndarray, V: int,
+              ignore_index: int = fi.IGNORE_INDEX, atol=LSE_ATOL):
+    """Rows in the loss: within `atol` of the oracle's logsumexp.  Rows outside it
+    (ignore_index, or a label outside [0, V)): exactly 0, as the library defines
+    (their logits are not computed)."""
+    labels = np.asarray(labels)
+    live = (labels != ignore_index) & (labels >= 0) & (labels < V)
+    assert np.all(np.asarray(got)[~live] == 0.0), "rows outside the loss must get lse 0"
+    if live.any():
+        err = np.abs(np.asarray(got, np.float64)[live] - np.asarray(ref)[live])
+        assert np.all(err <= atol), float(np.max(err - atol))
+
+
 def check_loss(got: float, ref: float):
     if ref == 0.0:
         assert got == 0.0, got

@@ -126,7 +126,7 @@ def test_options_host_side(lib):
                 "chunk_tokens": 16384, "chunk_vocab": 16384, "wait_timeout_ms": 1000,
                 "grad_tile_n": 512, "dz_tile_n": 256, "fwd_tile_n": 512, "fwd_group_m": 16,
                 "dz_group_m": 16, "grad_group_m": 8, "fwd_dynamic": 1,
-                "dz_buffers": 1}
+                "dz_buffers": 1, "fwd_compact": 1}
     assert set(defaults) == set(_native.OPTIONS)
     for name, dflt in defaults.items():
         assert _native.get_option(name) == dflt, name

@@ -35,7 +35,7 @@ def compare(got, hidden, weight, labels, softcap, reduction, grad_scale=1.0, gra
     assert got["loss_dtype"] == torch.float32
     assert got["ntok"] == rf["num_tokens"]
     G.check_loss(got["loss"], rf["loss"])
-    assert np.max(np.abs(got["lse"] - rf["lse"])) <= G.LSE_ATOL
+    G.check_lse(got["lse"], rf["lse"], labels, weight.shape[0], ignore_index)
     ign = labels == ignore_index
     assert np.all(got["dh"][ign] == 0.0), "ignored rows must get exact zero gradient"
     assert np.all(np.isfinite(got["dh"])) and np.all(np.isfinite(got["dw"]))
@@ -134,6 +134,14 @@ def test_label_out_of_range_is_reported():
         flce.forward(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
                      G.labels_tensor(y), check_status=True)
     assert e.value.status == 3
+    # the row is left out of the loss and the count, and its lse is 0, on every
+    # forward path
+    for compact in (1, 0):
+        with _native.options(fwd_compact=compact):
+            f = flce.forward(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
+                             G.labels_tensor(y))
+            torch.cuda.synchronize()
+        assert int(f.num_tokens.item()) == 129 and f.lse[5].item() == 0.0
     # the backward finds the same label on its own (compacted bf16, uncompacted, fp32)
     # and, like the forward, treats its row as ignored: the gradients equal, bit for
     # bit, those of the labels with that row set to ignore_index
@@ -335,6 +343,7 @@ def test_large_logits_stay_finite(softcap):
               G.labels_tensor(inp.labels), softcap, "sum")
     assert np.all(np.isfinite(got["lse"])) and np.isfinite(got["loss"])
     assert np.max(np.abs(got["lse"])) > (100.0 if softcap == 0 else 20.0)
+    live = inp.labels != IGN
     rf = oracle.forward(inp.hidden, inp.weight, inp.labels, IGN, softcap, "sum")
     rb = oracle.backward(inp.hidden, inp.weight, inp.labels, IGN, softcap, "sum")
     # lse: fp32 accumulation of K = 256 products errs by at most K * 2^-24 times the
@@ -342,7 +351,8 @@ def test_large_logits_stay_finite(softcap):
     # softcap only shrinks it
     absdot = np.abs(inp.hidden.astype(np.float64)) @ np.abs(inp.weight.astype(np.float64)).T
     tol = 256 * 2.0 ** -24 * absdot.max(axis=1) + G.LSE_ATOL
-    assert np.all(np.abs(got["lse"] - rf["lse"]) <= tol)
+    assert np.all(np.abs(got["lse"] - rf["lse"])[live] <= tol[live])
+    assert np.all(got["lse"][~live] == 0.0)
     G.check_loss(got["loss"], rf["loss"])
     assert got["ntok"] == rf["num_tokens"]
     assert np.all(got["dh"][inp.labels == IGN] == 0.0)
@@ -369,7 +379,7 @@ def test_degenerate_shapes(N, H, V, dtype):
         rf = oracle.forward(hid, wt, inp.labels, IGN, 0.0, "sum")
         assert got["ntok"] == rf["num_tokens"]
         assert abs(got["loss"]) <= 1e-5 * np.sum(np.abs(rf["lse"]))
-        assert np.max(np.abs(got["lse"] - rf["lse"])) <= G.LSE_ATOL
+        G.check_lse(got["lse"], rf["lse"], inp.labels, V)
         assert np.max(np.abs(got["dh"])) <= 1e-5 and np.max(np.abs(got["dw"])) <= 1e-5
     else:
         compare(got, hid, wt, inp.labels, 0.0, "sum")
@@ -379,14 +389,15 @@ def test_degenerate_shapes(N, H, V, dtype):
                                     "grad_tile_n=256", "dz_tile_n=512", "fwd_tile_n=256",
                                     "fwd_dynamic=0", "dz_buffers=2", "dz_buffers=2,bwd_fuse=0",
                                     "dz_buffers=2,cta_group=1", "fwd_group_m=3,dz_group_m=2,"
-                                    "grad_group_m=1"])
+                                    "grad_group_m=1", "fwd_compact=0", "fwd_compact=0,cta_group=1"])
 def test_alternative_paths(switch):
     """Each schedule option of the library selects another correct path: single-CTA
     128 x 256 tiles, separate dHidden and dWeight launches, no row compaction (and
     so no exact label term), 2-D views for MN-major operands, 256-column gradient
     and forward tiles, 512-column dZ tiles, round-robin forward tiles, two dZ
     blocks (9 chunks here, so a dZ launch waits on the gradient launches two
-    chunks back before it overwrites their block), other raster groups."""
+    chunks back before it overwrites their block), other raster groups, a
+    forward over every row instead of the compacted ones."""
     opts = {kv.split("=")[0]: int(kv.split("=")[1]) for kv in switch.split(",")}
     inp = G.small_inputs(N=2100, H=192, V=4500, seed=26, n_ign=300, w_std=0.1)
     with _native.options(**opts), G.chunks(*SMALL_CHUNKS):
@@ -495,3 +506,29 @@ def test_optional_gradients(dtype):
         assert W.grad is None
         # the same fp32 gradient (g = 1) rounded once to bf16: bit for bit
         assert torch.equal(hh.grad, ref_dh)
+
+
+@pytest.mark.parametrize("softcap,ign_frac", [(0.0, 0.3), (4.0, 0.95), (0.0, 1.0)])
+def test_forward_compaction_changes_no_bits(softcap, ign_frac):
+    """The forward's GEMM over the compacted rows computes each row's logits and
+    logsumexp in the same order as over all rows: lse bit-identical, the count
+    identical, the loss equal up to the order of its float64 sum; rows outside
+    the loss get lse 0 either way."""
+    N = 3000
+    inp = G.small_inputs(N=N, H=192, V=5000, seed=33, n_ign=int(ign_frac * N), w_std=0.1)
+    args = (G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
+            G.labels_tensor(inp.labels), IGN, softcap, "sum")
+    out = []
+    for compact in (1, 0):
+        with _native.options(fwd_compact=compact):
+            f = flce.forward(*args, check_status=True)
+            torch.cuda.synchronize()
+            out.append((f.loss.item(), int(f.num_tokens.item()), f.lse.cpu().numpy()))
+    (la, na, sa), (lb, nb, sb) = out
+    assert na == nb == int((inp.labels != IGN).sum())
+    assert np.array_equal(sa, sb)
+    assert abs(la - lb) <= 1e-6 * max(abs(lb), 1e-30)
+    assert np.all(sa[inp.labels == IGN] == 0.0)
+    rf = oracle.forward(inp.hidden, inp.weight, inp.labels, IGN, softcap, "sum")
+    G.check_loss(la, rf["loss"])
+    G.check_lse(sa, rf["lse"], inp.labels, 5000)
