@@ -1,16 +1,20 @@
 // Host side of the fused linear cross-entropy C ABI (include/flce.h):
 // argument checks, workspace layout, TMA tensor-map encoding and launches.
 //
-// bf16 path, forward:   tc_gemm<FwdStatsEpi> over all (128-token x 256-vocab)
-//                       tiles -> fwd_merge -> row_loss -> finalize.
-// bf16 path, backward:  the [N, V] problem is cut into chunks of at most
-//                       kChunkTokens x kChunkVocab; per chunk
+// bf16 path, forward:   row compaction (the rows in the loss first) ->
+//                       tc_gemm<FwdStatsEpi> over the valid rows' tiles ->
+//                       fwd_merge (lse back through the permutation) ->
+//                       row_loss -> finalize.
+// bf16 path, backward:  row compaction and label sort, then the [n, V]
+//                       problem is cut into chunks of at most chunk_tokens x
+//                       chunk_vocab (options); per chunk
 //                         tc_gemm<DzEpi>    dZ block (bf16, in the workspace)
 //                         tc_gemm<StoreEpi> (one launch, two GEMMs)
 //                           dHidden[chunk rows] (+)= dZ . W[chunk]
 //                           dWeight[chunk rows] (+)= dZ^T . hidden[chunk]
 //                       The first chunk along the reduced dimension stores,
-//                       later ones TMA-reduce-add into the fp32 outputs.
+//                       later ones add into the fp32 outputs; then the exact
+//                       fp32 label term of dWeight.
 // fp32 path:            simt_fwd / simt_dh / simt_dw (CUDA cores).
 #include <cuda.h>
 #include <cuda_runtime.h>

@@ -71,6 +71,6 @@ def small_inputs(N, H, V, seed, n_ign, w_std=0.05):
 
 def chunks(tokens: int, vocab: int):
     """Run the backward with tokens x vocab chunks instead of the default
-    8192 x 16384, so that small problems span several chunks along both
+    16384 x 16384, so that small problems span several chunks along both
     reduced dimensions (library options FLCE_OPT_CHUNK_TOKENS / _VOCAB)."""
     return _native.options(chunk_tokens=tokens, chunk_vocab=vocab)
