@@ -532,3 +532,14 @@ def test_forward_compaction_changes_no_bits(softcap, ign_frac):
     rf = oracle.forward(inp.hidden, inp.weight, inp.labels, IGN, softcap, "sum")
     G.check_loss(la, rf["loss"])
     G.check_lse(sa, rf["lse"], inp.labels, 5000)
+
+
+def test_two_token_chunks_at_the_default_chunk_size():
+    """N = 16384 + 300 rows cross the default 16384-token backward chunk: dWeight is
+    stored by the first token chunk and read-add-written by the second, with
+    512-column gradient tiles and the compacted passes; compared in full."""
+    N = 16384 + 300
+    inp = G.small_inputs(N=N, H=256, V=3000, seed=34, n_ign=N // 8, w_std=0.1)
+    got = run(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
+              G.labels_tensor(inp.labels), 0.0, "sum", grad_scale=1.0 / N)
+    compare(got, inp.hidden, inp.weight, inp.labels, 0.0, "sum", grad_scale=1.0 / N)

@@ -90,3 +90,27 @@ def test_two_streams_at_once():
     for got, ref in zip(outs, refs):
         for a, b in zip(got, ref):
             assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("buffers", [1, 2])
+def test_many_steps_back_to_back(buffers):
+    """Forty forward + backward steps enqueued without a host synchronisation in
+    between (so successive calls' dependent launches overlap on the device, and
+    with two dZ blocks the chunks' dZ and gradient launches overlap as well):
+    no bounded wait runs out and every step's results are bit-identical."""
+    h, W, y = _problem(35, N=3000, H=192, V=7000)
+    N, H = h.shape
+    V = W.shape[0]
+    with G.chunks(1024, 2048), _native.options(dz_buffers=buffers):
+        ref = _eager(h, W, y, 2.0)
+        ws = flce.alloc_workspace(N, H, V, torch.bfloat16, "cuda")
+        outs = []
+        for _ in range(40):
+            f = flce.forward(h, W, y, IGN, 2.0, "sum", workspace=ws)
+            dh, dw = flce.backward(h, W, y, f.lse, softcap=2.0, workspace=ws)
+            outs.append((f.loss, f.lse, dh, dw))
+        torch.cuda.synchronize()
+        assert flce.status(ws) == 0
+    for got in outs:
+        for a, b in zip(got, ref):
+            assert torch.equal(a, b)
