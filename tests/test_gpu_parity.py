@@ -543,3 +543,30 @@ def test_two_token_chunks_at_the_default_chunk_size():
     got = run(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
               G.labels_tensor(inp.labels), 0.0, "sum", grad_scale=1.0 / N)
     compare(got, inp.hidden, inp.weight, inp.labels, 0.0, "sum", grad_scale=1.0 / N)
+
+
+@pytest.mark.parametrize("width", [256, 512])
+def test_labels_at_tile_edges(width):
+    """Labels on both sides of every 256- and 512-column tile edge, the first and the
+    last vocabulary column of a ragged V, and an ignore_index inside the vocabulary
+    next to them: the label-logit capture and the label entry of dZ at the edges."""
+    V = 1283  # 5 x 256 + 3: the last tile holds 3 columns
+    edges = [0, 1, 254, 255, 256, 257, 510, 511, 512, 513, 767, 768, 1023, 1024, 1279, 1280,
+             V - 2, V - 1]
+    N = 4 * len(edges)
+    inp = G.small_inputs(N=N, H=136, V=V, seed=36, n_ign=0, w_std=0.3)
+    y = np.array(edges * 4, dtype=np.int64)
+    y[::9] = 1100  # the ignore_index below: a real vocabulary id
+    with _native.options(fwd_tile_n=width, dz_tile_n=width, grad_tile_n=width):
+        got = run(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
+                  G.labels_tensor(y), 2.5, "sum", ignore_index=1100)
+    compare(got, inp.hidden, inp.weight, y, 2.5, "sum", ignore_index=1100)
+
+
+def test_large_hidden_size():
+    """H = 8192 (the hidden size of 70B-class models): 128 K-blocks in the forward
+    and dZ GEMMs and 16 column tiles of 512 in dHidden and dWeight."""
+    inp = G.small_inputs(N=600, H=8192, V=3000, seed=37, n_ign=60, w_std=0.01)
+    got = run(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
+              G.labels_tensor(inp.labels), 0.0, "mean")
+    compare(got, inp.hidden, inp.weight, inp.labels, 0.0, "mean")
