@@ -13,8 +13,12 @@
 //                           dHidden[chunk rows] (+)= dZ . W[chunk]
 //                           dWeight[chunk rows] (+)= dZ^T . hidden[chunk]
 //                       The first chunk along the reduced dimension stores,
-//                       later ones add into the fp32 outputs; then the exact
-//                       fp32 label term of dWeight.
+//                       later ones add (TMA reduce-add) into fp32 outputs:
+//                       dWeight itself, and a compact-order dHidden block per
+//                       token chunk, which dh_scatter moves to token order
+//                       with the exact fp32 label term once the chunk's last
+//                       vocab chunk is done; at the end the exact fp32 label
+//                       term of dWeight.
 // fp32 path:            simt_fwd / simt_dh / simt_dw (CUDA cores).
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -331,10 +335,11 @@ int64_t bwd_counters(const Opts& o, int64_t N, int64_t V) { return 4 * bwd_chunk
 // compact labels and lse, per-block counts, valid count) | label sort (two
 // key/value buffers, digit counts) | label residuals | compact hidden [N, H]
 // bf16 | dZ block, whose space the dWeight label correction's run pieces
-// reuse once the GEMMs are done.
+// reuse once the GEMMs are done | compact-order dHidden of one token chunk
+// [chunk_tokens, H] fp32 (row compaction only).
 struct BwdLayout {
   size_t counters, perm, labels_c, lse_c, block_valid, n_valid_c, keys0, keys1, vals0, vals1,
-      hist, resid, hidden_c, gblock, gblock_bytes, part, end;
+      hist, resid, hidden_c, gblock, gblock_bytes, part, dh_c, end;
 };
 
 BwdLayout bwd_layout(const Opts& o, int64_t N, int64_t H, int64_t V) {
@@ -368,6 +373,9 @@ BwdLayout bwd_layout(const Opts& o, int64_t N, int64_t H, int64_t V) {
   const size_t nseg = static_cast<size_t>((N + kFixSeg - 1) / kFixSeg);
   off += std::max(L.gblock_bytes * static_cast<size_t>(o.dz_buffers),
                   nseg * 2 * static_cast<size_t>(H) * 4);
+  off = align_up(off, 1024);
+  L.dh_c = off;
+  if (o.compact) off += static_cast<size_t>(c.tc) * static_cast<size_t>(H) * 4;
   L.end = off;
   return L;
 }
@@ -806,13 +814,19 @@ flce_status backward_bf16(DevInfo* d, const Opts& o, const void* hidden, const v
     if (n_valid_is_count) n_valid = n_valid_c;  // the library's own count serves both
   }
 
+  // dHidden GEMM output: with row compaction a chunk-local compact-order fp32
+  // block (TMA stores and reduce-adds, then dh_scatter to token order),
+  // else d_hidden itself.
+  float* dh_c = compact ? reinterpret_cast<float*>(w + BL.dh_c) : nullptr;
+  float* dh_out = compact ? dh_c : d_hidden;
+  const int64_t dh_rows = compact ? ck.tc : N;
   CUtensorMap t_hid_k, t_hid_mn, t_w_k, t_w_mn, t_dh, t_dw;
   if (!make_map(&t_hid_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hid, H, N, H * 2, BK, BM) ||
       !make_map(&t_hid_mn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, hid, H, N, H * 2, 64, BK) ||
       !make_map(&t_w_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, weight, H, V, H * 2, BK, b_box_rows(o)) ||
       !make_map(&t_w_mn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, weight, H, V, H * 2, 64, BK) ||
-      (want_dh &&
-       !make_map(&t_dh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d_hidden, H, N, H * 4, 32, 32)) ||
+      (want_dh && !make_map(&t_dh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dh_out, H, dh_rows, H * 4,
+                            32, 32)) ||
       (want_dw &&
        !make_map(&t_dw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d_weight, H, V, H * 4, 32, 32)))
     return FLCE_ERR_CUDA;
@@ -910,13 +924,11 @@ flce_status backward_bf16(DevInfo* d, const Opts& o, const void* hidden, const v
       gh.dep_wait = kDepBeforeLoads;  // reads the dZ block written just before
       gh.b_mn3d = h3d ? 1 : 0;
       if (o.dz_buffers > 1) gh.done_counter = done + ci;
-      // the last vocab chunk's dHidden epilogue also adds the exact label term
       const bool last_v = v0 + ck.vc >= V;
-      StoreEpi::Params eh{static_cast<int>(t0), (v0 > 0 || acc_dh) ? 1 : 0, static_cast<int>(H),
-                          static_cast<int>(N), grad_output, grad_scale, n_valid, mean,
-                          perm, rows_valid, d_hidden, static_cast<int>(H),
-                          last_v ? resid : nullptr, lab,
-                          static_cast<const __nv_bfloat16*>(weight), static_cast<long long>(V)};
+      StoreEpi::Params eh{compact ? 0 : static_cast<int>(t0),
+                          (v0 > 0 || (acc_dh && !compact)) ? 1 : 0, static_cast<int>(H),
+                          compact ? rows : static_cast<int>(N), grad_output, grad_scale,
+                          n_valid, mean};
 
       // 3) dWeight[v0:v0+cols] (+)= dZ^T . hidden[t0:t0+rows]
       GemmArgs gw{};
@@ -937,8 +949,7 @@ flce_status backward_bf16(DevInfo* d, const Opts& o, const void* hidden, const v
       gw.b_mn3d = h3d ? 1 : 0;
       if (o.dz_buffers > 1) gw.done_counter = done + ci;
       StoreEpi::Params ew{static_cast<int>(v0), (t0 > 0 || acc_dw) ? 1 : 0, static_cast<int>(H),
-                          static_cast<int>(V), grad_output, grad_scale, n_valid, mean,
-                          nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0};
+                          static_cast<int>(V), grad_output, grad_scale, n_valid, mean};
 
       const GemmProblem ph{&t_g_k, &t_w_mn, &t_dh, rows, H, gh};
       const GemmProblem pw{&t_g_mn, &t_hid_mn, &t_dw, cols, H, gw};
@@ -960,6 +971,19 @@ flce_status backward_bf16(DevInfo* d, const Opts& o, const void* hidden, const v
         }
       }
       if (e != cudaSuccess) return cuda_fail(e);
+
+      if (compact && want_dh && last_v) {
+        // the token chunk's dHidden is complete: add the exact label term and
+        // move it to token order
+        e = launch(kHelper, st, [&] {
+          dh_scatter_kernel<<<rows, 256, 0, st>>>(
+              reinterpret_cast<const float4*>(dh_c), static_cast<int>(t0), rows, perm,
+              rows_valid, lab, resid, static_cast<const __nv_bfloat16*>(weight), V,
+              static_cast<int>(H / 4), reinterpret_cast<float4*>(d_hidden), acc_dh ? 1 : 0,
+              grad_output, grad_scale, n_valid, mean);
+        });
+        if (e != cudaSuccess) return cuda_fail(e);
+      }
     }
   }
 

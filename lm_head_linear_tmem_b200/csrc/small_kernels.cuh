@@ -555,6 +555,51 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// dHidden of one token chunk back to token order.  The chunk's dHidden GEMMs
+// accumulate g * dZ . W over the compact rows [t0, t0 + rows) into dh_c
+// (fp32, chunk-local rows, TMA store then reduce-add); here compact row j
+// adds the exact label term g * resid[j] * W[labels_c[j]] and lands on
+// d_hidden row perm[j] (stored, or added with `accumulate`).  Rows past the
+// valid count are not read: the GEMMs skip or leave them undefined.
+__global__ void __launch_bounds__(256)
+    dh_scatter_kernel(const float4* __restrict__ dh_c, int t0, int rows,
+                      const int* __restrict__ perm, const long long* __restrict__ n_valid,
+                      const int64_t* __restrict__ labels_c, const float* __restrict__ resid,
+                      const __nv_bfloat16* __restrict__ weight, int64_t V, int H4,
+                      float4* __restrict__ d_hidden, int accumulate, const float* grad_output,
+                      float grad_scale, const long long* n_valid_for_mean, int mean) {
+  const int jl = blockIdx.x;
+  const long long j = static_cast<long long>(t0) + jl;
+  if (jl >= rows || j >= *n_valid) return;
+  const float4* src = dh_c + static_cast<size_t>(jl) * H4;
+  float4* dst = d_hidden + static_cast<size_t>(perm[j]) * H4;
+  const int64_t y = labels_c[j];
+  const bool fix = resid != nullptr && y >= 0 && y < V;
+  const float cfix =
+      fix ? backward_grad_factor(grad_output, grad_scale, n_valid_for_mean, mean) * resid[j] : 0.f;
+  const uint2* wrow = reinterpret_cast<const uint2*>(weight + static_cast<size_t>(fix ? y : 0) * H4 * 4);
+  for (int k = threadIdx.x; k < H4; k += blockDim.x) {
+    float4 o = src[k];
+    if (fix) {
+      const uint2 wv = wrow[k];
+      const float2 w01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv.x));
+      const float2 w23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv.y));
+      o.x = fmaf(cfix, w01.x, o.x);
+      o.y = fmaf(cfix, w01.y, o.y);
+      o.z = fmaf(cfix, w23.x, o.z);
+      o.w = fmaf(cfix, w23.y, o.w);
+    }
+    if (accumulate) {
+      const float4 a = dst[k];
+      o.x += a.x;
+      o.y += a.y;
+      o.z += a.z;
+      o.w += a.w;
+    }
+    dst[k] = o;
+  }
+}
+
 // Waits, bounded, on an mbarrier that nothing completes; records the timeout
 // in the status word (the same wait and report as the GEMM pipelines).
 __global__ void selftest_wait_kernel(unsigned int* status, unsigned long long timeout_ns) {

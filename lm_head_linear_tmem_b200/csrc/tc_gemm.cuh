@@ -347,16 +347,6 @@ struct StoreEpi {
     float grad_scale;
     const long long* n_valid;  // device count of non-ignored rows
     int mean;
-    const int* row_map;          // scatter mode: compact row -> output row
-    const long long* rows_valid; // scatter mode: rows that exist
-    float* out_ptr;              // scatter mode: output base
-    int ld;                      // scatter mode: output row stride (floats)
-    // scatter mode, dHidden: adds g * resid[r] * W[labels[r]] to row r (the
-    // exact label term; see DzEpi).  Null for no correction.
-    const float* fix_resid;
-    const int64_t* fix_labels;
-    const __nv_bfloat16* fix_w;  // [V, x_limit] row-major
-    long long fix_v;
   };
 
   __device__ static float grad_factor(const Params& p) {
@@ -373,11 +363,9 @@ struct StoreEpi {
                               const CUtensorMap* out, uint32_t tempty, int& nstore,
                               bool empty) {
     const int y = p.out_row0 + m_base + q * 32;
-    int y_end = p.y_limit;
-    if (p.row_map != nullptr) y_end = static_cast<int>(min(static_cast<long long>(y_end), *p.rows_valid));
     // 32-column chunks whose store box starts inside the output (warp-uniform)
     const int rem = p.x_limit - col0;
-    const int nch = (y >= y_end || rem <= 0) ? 0 : min(BN / 32, (rem + 31) / 32);
+    const int nch = (y >= p.y_limit || rem <= 0) ? 0 : min(BN / 32, (rem + 31) / 32);
     if (nch == 0) {
       release_tmem(tempty, lane);
       return;
@@ -385,58 +373,6 @@ struct StoreEpi {
     // An empty K range contributes zeros: the accumulator was never written, so
     // its stale contents are not read (0 * stale could be NaN).
     const float g = empty ? 0.0f : grad_factor(p);
-    if (p.row_map != nullptr) {
-      const int r = y + lane;
-      const bool live = r < y_end;
-      float* dst = p.out_ptr + static_cast<size_t>(live ? p.row_map[r] : 0) * p.ld + col0;
-      float cfix = 0.f;
-      const __nv_bfloat16* wrow = nullptr;
-      if (p.fix_resid != nullptr && live && !empty) {
-        const int64_t yl = p.fix_labels[r];
-        if (yl >= 0 && yl < p.fix_v) {
-          cfix = g * p.fix_resid[r];
-          wrow = p.fix_w + static_cast<size_t>(yl) * p.x_limit + col0;
-        }
-      }
-#pragma unroll 1
-      for (int c = 0; c < nch; ++c) {
-        uint32_t v[32];
-        tmem_ld_x32(taddr + c * 32, v);
-        tmem_ld_wait();
-        if (c == nch - 1) release_tmem(tempty, lane);
-        if (empty) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = 0u;
-        }
-        if (live) {
-#pragma unroll
-          for (int j4 = 0; j4 < 8; ++j4) {
-            if (col0 + c * 32 + 4 * j4 >= p.x_limit) break;  // x_limit is a multiple of 4
-            float4 o = make_float4(__uint_as_float(v[4 * j4]) * g, __uint_as_float(v[4 * j4 + 1]) * g,
-                                   __uint_as_float(v[4 * j4 + 2]) * g, __uint_as_float(v[4 * j4 + 3]) * g);
-            float4* d4 = reinterpret_cast<float4*>(dst + c * 32) + j4;
-            if (wrow != nullptr) {
-              const uint2 wv = *reinterpret_cast<const uint2*>(wrow + c * 32 + 4 * j4);
-              const float2 w01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv.x));
-              const float2 w23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv.y));
-              o.x = fmaf(cfix, w01.x, o.x);
-              o.y = fmaf(cfix, w01.y, o.y);
-              o.z = fmaf(cfix, w23.x, o.z);
-              o.w = fmaf(cfix, w23.y, o.w);
-            }
-            if (p.reduce) {
-              const float4 a = *d4;
-              o.x += a.x;
-              o.y += a.y;
-              o.z += a.z;
-              o.w += a.w;
-            }
-            *d4 = o;
-          }
-        }
-      }
-      return;
-    }
     const uint32_t stg_u32 = smem_u32(stg);
 #pragma unroll 1
     for (int c = 0; c < nch; ++c) {

@@ -57,8 +57,11 @@ def test_workspace_bytes(lib):
     big = ws(16384, 4096, 131072, 0)
     # forward partials: 512 vocab tiles x 16384 rows x (m, s) fp32 = 64 MiB;
     # backward: compact hidden 16384 x 4096 bf16 = 128 MiB + dZ block
-    # 16384 x 16384 bf16 = 512 MiB + row-compaction, label-sort and residual arrays
-    assert 640 * 2 ** 20 <= big < 642 * 2 ** 20
+    # 16384 x 16384 bf16 = 512 MiB + compact-order dHidden of a token chunk
+    # 16384 x 4096 fp32 = 256 MiB + row-compaction, label-sort and residual arrays
+    assert 896 * 2 ** 20 <= big < 898 * 2 ** 20
+    with _native.options(bwd_compact=0):  # dHidden goes straight to its output
+        assert ws(16384, 4096, 131072, 0) <= big - 256 * 2 ** 20
     assert ws(0, 64, 512, 0) > 0
     assert ws(64, 64, 512, 1) > 0
     ex = lib.flce_workspace_bytes_ex
