@@ -106,9 +106,10 @@ typedef enum flce_option {
   FLCE_OPT_MN3D = 3,            /* [1] MN-major operands load through 3-D chunk views; 0: 2-D views */
   FLCE_OPT_CHUNK_TOKENS = 4,    /* [16384] token rows of a backward chunk (256 .. 2^20, rounded up to 256) */
   FLCE_OPT_CHUNK_VOCAB = 5,     /* [16384] vocab columns of a backward chunk (256 .. 2^20, rounded up to 256);
-                                   the dZ block of the workspace is chunk_tokens x chunk_vocab bf16, so
-                                   flce_workspace_bytes must be called with the same chunk options as the
-                                   calls that use the workspace */
+                                   the dZ block of the workspace is chunk_tokens x chunk_vocab bf16 and,
+                                   with FLCE_OPT_BWD_COMPACT, a compact-order dHidden block chunk_tokens x H
+                                   fp32 follows it, so flce_workspace_bytes must be called with the same
+                                   chunk and compaction options as the calls that use the workspace */
   FLCE_OPT_WAIT_TIMEOUT_MS = 6, /* [1000] limit of every bounded wait inside a kernel (10 .. 60000) */
   FLCE_OPT_GRAD_TILE_N = 7,     /* [512] columns of a dHidden / dWeight tile: 512 or 256 (512 needs CTA pairs;
                                    with FLCE_OPT_CTA_GROUP = 1 tiles are 256 wide) */
