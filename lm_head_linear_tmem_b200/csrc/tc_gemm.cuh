@@ -43,6 +43,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <type_traits>
 #include <math_constants.h>
 
 #include "ptx.cuh"
@@ -179,7 +180,16 @@ struct FwdStatsEpi {
     float* label_logit;  // [N]
   };
 
-  __device__ static void tile(const Params& p, const GemmArgs&, int m_base, int col0,
+  // The row's label, read before the accumulator is ready.
+  struct Pre {
+    int64_t y;
+  };
+  __device__ static Pre prepare(const Params& p, int m_base, int q, int lane) {
+    const int row = m_base + q * 32 + lane;
+    return Pre{row < p.N ? p.labels[row] : int64_t{-1}};
+  }
+
+  __device__ static void tile(const Params& p, const Pre& pre, int m_base, int col0,
                               uint32_t taddr, int q, int lane, uint8_t*, const CUtensorMap*,
                               uint32_t tempty, int&, bool) {
     if (col0 >= p.V) {  // the second bank of a 512-column tile past the vocabulary
@@ -190,37 +200,64 @@ struct FwdStatsEpi {
     const bool row_ok = row < p.N;
     const int nb = col0 / BN;
     int y_local = -1;
-    if (row_ok) {
-      const int64_t y = p.labels[row];
-      if (y >= col0 && y < static_cast<int64_t>(col0) + BN) y_local = static_cast<int>(y - col0);
-    }
+    if (row_ok && pre.y >= col0 && pre.y < static_cast<int64_t>(col0) + BN)
+      y_local = static_cast<int>(pre.y - col0);
     const int ncols = min(BN, p.V - col0);
-    float m = -CUDART_INF_F;
+    // warp-uniform: does any row's label fall in this bank?
+    const bool any_label = __any_sync(0xffffffffu, y_local >= 0);
+    float m = -CUDART_INF_F;  // log2 domain
     float s = 0.f;
     float ly = 0.f;
-#pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-      uint32_t r[32];
-      tmem_ld_x32(taddr + c * 32, r);
-      tmem_ld_wait();
-      if (c == BN / 32 - 1) release_tmem(tempty, lane);
-      float t[32];
-      float cmax = -CUDART_INF_F;
+    // 32-column chunks, the next chunk's TMEM load in flight while this one is
+    // reduced; max as a tree, sum of exp2 over four partial sums
+    auto chunk = [&](int c, const uint32_t(&r)[32]) {
+      float L[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const float z = __uint_as_float(r[j]);
-        const float L = kSoftcap ? p.softcap * tanhf(z * p.inv_softcap) : z;
-        const int col = c * 32 + j;
-        if (col == y_local) ly = L;
-        t[j] = (col < ncols) ? L * kLog2e : -CUDART_INF_F;
-        cmax = fmaxf(cmax, t[j]);
+        L[j] = kSoftcap ? p.softcap * tanhf(z * p.inv_softcap) : z;
       }
-      const float mn = fmaxf(m, cmax);
-      float acc = 0.f;
+      if (any_label) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) acc += exp2f(t[j] - mn);
-      s = (m == -CUDART_INF_F) ? acc : s * exp2f(m - mn) + acc;
+        for (int j = 0; j < 32; ++j)
+          if (c * 32 + j == y_local) ly = L[j];
+      }
+      if (c * 32 + 32 > ncols) {  // the vocabulary ends inside this chunk
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (c * 32 + j >= ncols) L[j] = -CUDART_INF_F;
+      }
+      float mx[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) mx[j] = fmaxf(L[j], L[j + 16]);
+#pragma unroll
+      for (int w = 8; w >= 1; w /= 2)
+#pragma unroll
+        for (int j = 0; j < w; ++j) mx[j] = fmaxf(mx[j], mx[j + w]);
+      const float mn = fmaxf(m, mx[0] * kLog2e);
+      float a4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int j = 0; j < 32; ++j) a4[j & 3] += ex2_approx(fmaf(L[j], kLog2e, -mn));
+      const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+      s = (m == -CUDART_INF_F) ? acc : fmaf(s, ex2_approx(m - mn), acc);
       m = mn;
+    };
+    // chunks in pairs, even ones from buf[0], odd ones from buf[1]; the
+    // softcapped body (a tanh per logit) is kept rolled to bound code size
+    uint32_t buf[2][32];
+    tmem_ld_x32(taddr, buf[0]);
+    tmem_ld_wait(buf[0]);
+#pragma unroll(kSoftcap ? 1 : BN / 64)
+    for (int c = 0; c < BN / 32; c += 2) {
+      tmem_ld_x32(taddr + (c + 1) * 32, buf[1]);
+      chunk(c, buf[0]);
+      tmem_ld_wait(buf[1]);
+      if (c + 2 < BN / 32)
+        tmem_ld_x32(taddr + (c + 2) * 32, buf[0]);
+      else
+        release_tmem(tempty, lane);  // every column of the bank is in registers
+      chunk(c + 1, buf[1]);
+      if (c + 2 < BN / 32) tmem_ld_wait(buf[0]);
     }
     if (row_ok) {
       const size_t idx = static_cast<size_t>(nb) * p.N + row;
@@ -259,7 +296,18 @@ struct DzEpi {
     int64_t v_total;   // V: a label outside [0, V) counts as ignored
   };
 
-  __device__ static void tile(const Params& p, const GemmArgs&, int m_base, int col0,
+  // The row's label and lse, read before the accumulator is ready.
+  struct Pre {
+    int64_t y;
+    float lse;
+  };
+  __device__ static Pre prepare(const Params& p, int m_base, int q, int lane) {
+    const int row_l = m_base + q * 32 + lane;
+    if (row_l >= p.rows) return Pre{0, 0.f};
+    return Pre{p.labels[p.t0 + row_l], p.lse[p.t0 + row_l]};
+  }
+
+  __device__ static void tile(const Params& p, const Pre& pre, int m_base, int col0,
                               uint32_t taddr, int q, int lane, uint8_t* stg,
                               const CUtensorMap* out, uint32_t tempty, int& nstore, bool) {
     // 64-column chunks whose store box starts inside the block (warp-uniform)
@@ -275,57 +323,88 @@ struct DzEpi {
     int y_local = -1;
     float lse2 = 0.f;
     if (row_l < p.rows) {
-      const int row = p.t0 + row_l;
-      const int64_t y = p.labels[row];
+      const int64_t y = pre.y;
       valid = (y != p.ignore_index) && y >= 0 && y < p.v_total;
       const int64_t c0 = static_cast<int64_t>(p.v0) + col0;
       if (valid && y >= c0 && y < c0 + BN) y_local = static_cast<int>(y - c0);
-      lse2 = p.lse[row] * kLog2e;
+      lse2 = pre.lse * kLog2e;
     }
     const uint32_t stg_u32 = smem_u32(stg);
-#pragma unroll 1
-    for (int c2 = 0; c2 < nch; ++c2) {
-      uint32_t r0[32], r1[32];
-      tmem_ld_x32(taddr + c2 * 64, r0);
-      tmem_ld_x32(taddr + c2 * 64 + 32, r1);
-      tmem_ld_wait();
-      if (c2 == nch - 1) release_tmem(tempty, lane);
-      uint32_t packed[32];
+    // warp-uniform: does any row's label fall in this bank?
+    const bool any_label = __any_sync(0xffffffffu, y_local >= 0);
+    // 32-column sub-chunks, the next one's TMEM load in flight while this one
+    // is computed; every 64 columns are staged and stored
+    uint32_t packed[32];
+    // sub-chunk sc (32 columns) into half kH of `packed`; the odd half stages
+    // and stores the 64 columns
+    auto sub = [&](int sc, const uint32_t(&r)[32], auto half) {
+      constexpr int kH = decltype(half)::value;
+      if (sc >= 2 * nch) return;
+      float d[32], f[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        float gv[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int jj = 2 * j + h;
-          const float z = __uint_as_float(jj < 32 ? r0[jj] : r1[jj - 32]);
-          const float L = kSoftcap ? p.softcap * tanhf(z * p.inv_softcap) : z;
-          float d = exp2f(fmaf(L, kLog2e, -lse2));
-          if (c2 * 64 + jj == y_local) d -= 1.0f;
-          if (kSoftcap) {
-            const float u = L * p.inv_softcap;
-            d *= fmaf(-u, u, 1.0f);
-          }
-          if (p.resid != nullptr && c2 * 64 + jj == y_local)
-            p.resid[p.t0 + row_l] = d - __bfloat162float(__float2bfloat16_rn(d));
-          gv[h] = valid ? d : 0.0f;
+        const float z = __uint_as_float(r[j]);
+        const float L = kSoftcap ? p.softcap * tanhf(z * p.inv_softcap) : z;
+        d[j] = ex2_approx(fmaf(L, kLog2e, -lse2));
+        if (kSoftcap) {
+          const float u = L * p.inv_softcap;
+          f[j] = fmaf(-u, u, 1.0f);
         }
-        __nv_bfloat162 b2 = __floats2bfloat162_rn(gv[0], gv[1]);
-        packed[j] = *reinterpret_cast<uint32_t*>(&b2);
       }
-      // Buffer = parity of this warp's store count: the store that last read
-      // this buffer is the one before the most recent, which wait_read<1>
-      // has retired.
-      const int b = nstore & 1;
-      if (lane == 0) bulk_wait_group_read<1>();
-      __syncwarp();
-      stage_row_128b(stg + b * kStagingBuf, lane, packed);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        tma_store_2d(out, stg_u32 + b * kStagingBuf, col0 + c2 * 64, y0);
-        bulk_commit_group();
+      if (any_label) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (sc * 32 + j == y_local) d[j] -= 1.0f;
       }
-      ++nstore;
+      if (kSoftcap) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) d[j] *= f[j];
+      }
+      if (any_label && p.resid != nullptr) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (sc * 32 + j == y_local)
+            p.resid[p.t0 + row_l] = d[j] - __bfloat162float(__float2bfloat16_rn(d[j]));
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        __nv_bfloat162 b2 =
+            __floats2bfloat162_rn(valid ? d[2 * j] : 0.0f, valid ? d[2 * j + 1] : 0.0f);
+        packed[kH * 16 + j] = *reinterpret_cast<uint32_t*>(&b2);
+      }
+      if (kH == 1) {
+        // Buffer = parity of this warp's store count: the store that last
+        // read this buffer is the one before the most recent, which
+        // wait_read<1> has retired.
+        const int b = nstore & 1;
+        if (lane == 0) bulk_wait_group_read<1>();
+        __syncwarp();
+        stage_row_128b(stg + b * kStagingBuf, lane, packed);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(out, stg_u32 + b * kStagingBuf, col0 + (sc >> 1) * 64, y0);
+          bulk_commit_group();
+        }
+        ++nstore;
+      }
+    };
+    // sub-chunks in pairs (one 64-column store each), the next one's TMEM load
+    // in flight while one is computed; the softcapped body stays rolled
+    uint32_t buf[2][32];
+    tmem_ld_x32(taddr, buf[0]);
+    tmem_ld_wait(buf[0]);
+#pragma unroll(kSoftcap ? 1 : BN / 64)
+    for (int sc = 0; sc < BN / 32; sc += 2) {
+      tmem_ld_x32(taddr + (sc + 1) * 32, buf[1]);
+      sub(sc, buf[0], std::integral_constant<int, 0>{});
+      tmem_ld_wait(buf[1]);
+      if (sc + 2 < BN / 32)
+        tmem_ld_x32(taddr + (sc + 2) * 32, buf[0]);
+      else
+        release_tmem(tempty, lane);  // every column of the bank is in registers
+      sub(sc + 1, buf[1], std::integral_constant<int, 1>{});
+      if (sc + 2 < BN / 32) tmem_ld_wait(buf[0]);
     }
   }
 };
@@ -334,9 +413,6 @@ struct DzEpi {
 // Tile * g -> fp32 output rows [out_row0 + m]: TMA store, or TMA reduce-add
 // when `reduce` (accumulation across chunks of the split reduction dimension).
 // g = grad_output * grad_scale, divided by max(n, 1) for 'mean'.
-// With row_map set, output row r is row row_map[r] of out_ptr (row stride ld)
-// and only rows r < *rows_valid exist: the tile is written with vector stores
-// (reduce: read, add, write; each element has one writer per launch).
 struct StoreEpi {
   struct Params {
     int out_row0;
@@ -358,7 +434,13 @@ struct StoreEpi {
     return g;
   }
 
-  __device__ static void tile(const Params& p, const GemmArgs&, int m_base, int col0,
+  // The scale g, read before the accumulator is ready.
+  struct Pre {
+    float g;
+  };
+  __device__ static Pre prepare(const Params& p, int, int, int) { return Pre{grad_factor(p)}; }
+
+  __device__ static void tile(const Params& p, const Pre& pre, int m_base, int col0,
                               uint32_t taddr, int q, int lane, uint8_t* stg,
                               const CUtensorMap* out, uint32_t tempty, int& nstore,
                               bool empty) {
@@ -372,7 +454,7 @@ struct StoreEpi {
     }
     // An empty K range contributes zeros: the accumulator was never written, so
     // its stale contents are not read (0 * stale could be NaN).
-    const float g = empty ? 0.0f : grad_factor(p);
+    const float g = empty ? 0.0f : pre.g;
     const uint32_t stg_u32 = smem_u32(stg);
 #pragma unroll 1
     for (int c = 0; c < nch; ++c) {
@@ -844,6 +926,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok || tile >= num_tiles) break;
       int prob, mb, nb;
       locate(tile, prob, mb, nb);
+      const int m_base = mb * Cfg::kUnitRows + static_cast<int>(rank) * BM;
+      const GemmArgs& ga = prob ? a1 : a0;
+      // per-row inputs of the epilogue, in flight while the MMAs finish
+      const typename Epi::Pre pre = Epi::prepare(prob ? ep1 : ep0, m_base, q, lane);
       // the tile's first bank and the phase its full barrier completes
       const uint32_t acc = (kBanks == 1) ? (it & 1) : 0u;
       const uint32_t aph = (kBanks == 1) ? ((it >> 1) & 1) : (it & 1);
@@ -854,15 +940,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int m_base = mb * Cfg::kUnitRows + static_cast<int>(rank) * BM;
-      const GemmArgs& ga = prob ? a1 : a0;
 #pragma unroll 1
       for (int h = 0; h < kBanks; ++h) {  // bank 0 first: the next tile starts on it
         const uint32_t bank = acc + h;
         const uint32_t taddr = tmem_base + bank * BN + (static_cast<uint32_t>(q * 32) << 16);
         const uint32_t tempty_local = smem_u32(&bar_tempty[bank]);
         const uint32_t tempty = (kCG == 1) ? tempty_local : mapa_shared(tempty_local, 0);
-        Epi::tile(prob ? ep1 : ep0, ga, m_base, nb * kBN + h * BN, taddr, q, lane, stg,
+        Epi::tile(prob ? ep1 : ep0, pre, m_base, nb * kBN + h * BN, taddr, q, lane, stg,
                   prob ? &tmOut1 : &tmOut0, tempty, nstore, ga.k_blocks == 0);
       }
     }
