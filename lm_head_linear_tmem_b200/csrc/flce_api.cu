@@ -484,7 +484,9 @@ cudaError_t run_gemm_cg(DevInfo* d, int kind, const GemmProblem& p0,
                         const typename Epi::Params& ep1, cudaStream_t st, int* ctas_out) {
   using Cfg = TileCfg<kCG, kBN>;
   auto k = tc_gemm_kernel<Epi, kCG, kBN, kAMn0, kBMn0, kAMn1, kBMn1>;
-  cudaError_t e = set_smem_attr(k, Cfg::kSmemBytes);
+  constexpr size_t kSmem = gemm_smem_bytes<Epi, kCG, kBN>();
+  static_assert(kSmem <= 227 * 1024 - 512, "shared memory");
+  cudaError_t e = set_smem_attr(k, kSmem);
   if (e != cudaSuccess) return e;
   GemmArgs g0 = p0.g;
   g0.m_tiles = static_cast<int>((p0.M + Cfg::kUnitRows - 1) / Cfg::kUnitRows);
@@ -502,8 +504,8 @@ cudaError_t run_gemm_cg(DevInfo* d, int kind, const GemmProblem& p0,
   if (ctas_out != nullptr) *ctas_out = units * kCG;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(units * kCG, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.blockDim = dim3(gemm_threads<Epi>(), 1, 1);
+  cfg.dynamicSmemBytes = kSmem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   int nattr = 0;

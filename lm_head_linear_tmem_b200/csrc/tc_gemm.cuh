@@ -1,11 +1,14 @@
 // Persistent tcgen05 GEMM for the fused linear cross-entropy (FLCE).
 //
-// One CTA per SM (192 threads, ~225 KB shared memory, all 512 TMEM columns).
-// Warp roles:
+// One CTA per SM (192 or 320 threads, up to ~225 KB shared memory, all 512
+// TMEM columns).  Warp roles:
 //   warp 0  TMA producer   (one thread): K-blocks of A and B into a stage ring
 //   warp 1  MMA issuer     (one thread): tcgen05.mma K=16 steps, fp32 in TMEM
-//   warps 2-5 epilogue     (128 threads, thread = accumulator row): tcgen05.ld
-//                                        then an operation-specific epilogue
+//   warps 2.. epilogue     4 or 8 warps (a trait of the epilogue), thread =
+//                          accumulator row: tcgen05.ld then an operation-
+//                          specific epilogue.  A warp may read only its TMEM
+//                          lane quadrant (warp % 4); with 8 warps two share a
+//                          quadrant and each takes half of a bank's columns.
 // Tile shapes (template parameters kCG, the CTA group, and kBN, the columns of
 // a tile):
 //   kCG = 1, kBN = 256  one CTA computes a 128 x 256 tile
@@ -54,10 +57,8 @@ constexpr int BM = 128;  // accumulator rows held by one CTA
 constexpr int BN = 256;  // accumulator columns
 constexpr int BK = 64;
 constexpr int kABytes = BM * BK * 2;  // 16 KB
-constexpr int kEpiWarps = 4;
 constexpr int kStagingBuf = 4096;                 // 32 rows x 128 bytes
-constexpr int kStagingPerWarp = 2 * kStagingBuf;  // double buffered
-constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kStagingPerWarp = 2 * kStagingBuf;  // double buffered (TMA-store epilogues)
 constexpr uint32_t kTmemCols = 512;
 
 template <int kCG, int kBN = 256>
@@ -71,10 +72,20 @@ struct TileCfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStages = (kCG == 1 || kBN == 512) ? 4 : 6;
   static constexpr int kUnitRows = BM * kCG;  // output rows of one tile
-  static constexpr size_t kSmemBytes =
-      1024 + static_cast<size_t>(kStages) * kStageBytes + kEpiWarps * kStagingPerWarp;
-  static_assert(kSmemBytes <= 227 * 1024 - 512, "shared memory");
+  static constexpr size_t kRingBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes;
 };
+
+// Threads and dynamic shared memory of a GEMM CTA with epilogue Epi (its
+// warps and per-warp staging bytes are traits of the epilogue).
+template <class Epi>
+constexpr int gemm_threads() {
+  return 64 + 32 * Epi::kEpiWarps;
+}
+template <class Epi, int kCG, int kBN>
+constexpr size_t gemm_smem_bytes() {
+  return TileCfg<kCG, kBN>::kRingBytes +
+         static_cast<size_t>(Epi::kEpiWarps) * Epi::kStagingPerWarp;
+}
 
 constexpr int kRing = 8;  // tile indices in flight between the fetcher and the other roles
 
@@ -167,8 +178,22 @@ __device__ __forceinline__ void stage_row_128b(uint8_t* buf, int lane, const uin
 // Per tile: L = softcap(Z) over 256 vocab columns; per row the maximum m and
 // s = sum exp(L - m) (both in the log2 domain), written to partials
 // [n_tile][N]; the label logit L[i, y_i] is written by the tile holding y_i.
+// Eight epilogue warps: the two warps of a TMEM lane quadrant each reduce 128
+// of the bank's columns, and the second hands its (m, s) to the first through
+// shared memory (two slots used in turn, each with a full and an empty
+// mbarrier; bounded waits), which merges and writes them.
 template <bool kSoftcap>
 struct FwdStatsEpi {
+  static constexpr int kEpiWarps = 8;
+  // first warp of a quadrant: its mbarriers full[2], empty[2]; second warp:
+  // the two (m[32], s[32]) slots
+  static constexpr int kStagingPerWarp = 2 * 64 * 4;
+  __device__ static void init_smem(uint8_t* staging) {
+    for (int w = 0; w < 4; ++w) {
+      uint64_t* b = reinterpret_cast<uint64_t*>(staging + w * kStagingPerWarp);
+      for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&b[i]), 1);
+    }
+  }
   struct Params {
     const int64_t* labels;
     int N;
@@ -189,82 +214,146 @@ struct FwdStatsEpi {
     return Pre{row < p.N ? p.labels[row] : int64_t{-1}};
   }
 
-  __device__ static void tile(const Params& p, const Pre& pre, int m_base, int col0,
-                              uint32_t taddr, int q, int lane, uint8_t*, const CUtensorMap*,
-                              uint32_t tempty, int&, bool) {
+  __device__ static bool tile(const Params& p, const Pre& pre, int m_base, int col0,
+                              uint32_t taddr, int q, int lane, int part, uint8_t* stg,
+                              const CUtensorMap*, uint32_t tempty, int& nbank, bool,
+                              const volatile int* abort, unsigned long long timeout_ns) {
     if (col0 >= p.V) {  // the second bank of a 512-column tile past the vocabulary
       release_tmem(tempty, lane);
-      return;
+      return true;
     }
+    const int slot = nbank & 1;
+    const uint32_t use = static_cast<uint32_t>(nbank >> 1);  // earlier uses of this slot
+    ++nbank;
     const int row = m_base + q * 32 + lane;
     const bool row_ok = row < p.N;
-    const int nb = col0 / BN;
+    const int h0 = col0 + part * (BN / 2);  // this warp's first column
     int y_local = -1;
-    if (row_ok && pre.y >= col0 && pre.y < static_cast<int64_t>(col0) + BN)
-      y_local = static_cast<int>(pre.y - col0);
-    const int ncols = min(BN, p.V - col0);
-    // warp-uniform: does any row's label fall in this bank?
+    if (row_ok && pre.y >= h0 && pre.y < static_cast<int64_t>(h0) + BN / 2)
+      y_local = static_cast<int>(pre.y - h0);
+    const int ncols = max(0, min(BN / 2, p.V - h0));
+    // warp-uniform: does any row's label fall in these columns?
     const bool any_label = __any_sync(0xffffffffu, y_local >= 0);
     float m = -CUDART_INF_F;  // log2 domain
     float s = 0.f;
     float ly = 0.f;
-    // 32-column chunks, the next chunk's TMEM load in flight while this one is
-    // reduced; max as a tree, sum of exp2 over four partial sums
-    auto chunk = [&](int c, const uint32_t(&r)[32]) {
-      float L[32];
+    const uint32_t ta = taddr + part * (BN / 2);
+    if constexpr (!kSoftcap) {
+      // all 128 columns into registers, the TMEM half released at once (the
+      // next tile's MMAs wait for it), then one max and one sum over them
+      uint32_t r[4][32];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float z = __uint_as_float(r[j]);
-        L[j] = kSoftcap ? p.softcap * tanhf(z * p.inv_softcap) : z;
-      }
+      for (int c = 0; c < 4; ++c) tmem_ld_x32(ta + c * 32, r[c]);
+      tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) reg_fence(r[c]);
+      release_tmem(tempty, lane);
       if (any_label) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (c * 32 + j == y_local) ly = L[j];
+        for (int j = 0; j < 128; ++j)
+          if (j == y_local) ly = __uint_as_float(r[j / 32][j % 32]);
       }
-      if (c * 32 + 32 > ncols) {  // the vocabulary ends inside this chunk
+      if (ncols < BN / 2) {  // the vocabulary ends inside (or before) these columns
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (c * 32 + j >= ncols) L[j] = -CUDART_INF_F;
+        for (int j = 0; j < 128; ++j)
+          if (j >= ncols) r[j / 32][j % 32] = __float_as_uint(-CUDART_INF_F);
       }
-      float mx[16];
+      float mx[32];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) mx[j] = fmaxf(L[j], L[j + 16]);
+      for (int j = 0; j < 32; ++j)
+        mx[j] = fmaxf(fmaxf(__uint_as_float(r[0][j]), __uint_as_float(r[1][j])),
+                      fmaxf(__uint_as_float(r[2][j]), __uint_as_float(r[3][j])));
 #pragma unroll
-      for (int w = 8; w >= 1; w /= 2)
+      for (int w = 16; w >= 1; w /= 2)
 #pragma unroll
         for (int j = 0; j < w; ++j) mx[j] = fmaxf(mx[j], mx[j + w]);
-      const float mn = fmaxf(m, mx[0] * kLog2e);
-      float a4[4] = {0.f, 0.f, 0.f, 0.f};
+      if (mx[0] != -CUDART_INF_F) {
+        m = mx[0] * kLog2e;
+        float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j = 0; j < 32; ++j) a4[j & 3] += ex2_approx(fmaf(L[j], kLog2e, -mn));
-      const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
-      s = (m == -CUDART_INF_F) ? acc : fmaf(s, ex2_approx(m - mn), acc);
-      m = mn;
-    };
-    // chunks in pairs, even ones from buf[0], odd ones from buf[1]; the
-    // softcapped body (a tanh per logit) is kept rolled to bound code size
-    uint32_t buf[2][32];
-    tmem_ld_x32(taddr, buf[0]);
-    tmem_ld_wait(buf[0]);
-#pragma unroll(kSoftcap ? 1 : BN / 64)
-    for (int c = 0; c < BN / 32; c += 2) {
-      tmem_ld_x32(taddr + (c + 1) * 32, buf[1]);
-      chunk(c, buf[0]);
-      tmem_ld_wait(buf[1]);
-      if (c + 2 < BN / 32)
-        tmem_ld_x32(taddr + (c + 2) * 32, buf[0]);
-      else
-        release_tmem(tempty, lane);  // every column of the bank is in registers
-      chunk(c + 1, buf[1]);
-      if (c + 2 < BN / 32) tmem_ld_wait(buf[0]);
+        for (int j = 0; j < 128; ++j)
+          a8[j & 7] += ex2_approx(fmaf(__uint_as_float(r[j / 32][j % 32]), kLog2e, -m));
+        s = ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
+      }
+    } else {
+      // softcapped: 32-column chunks with an online max, the next chunk's
+      // TMEM load in flight; the tanh body is kept rolled to bound code size
+      auto chunk = [&](int c, const uint32_t(&r)[32]) {
+        float L[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) L[j] = p.softcap * tanhf(__uint_as_float(r[j]) * p.inv_softcap);
+        if (any_label) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (c * 32 + j == y_local) ly = L[j];
+        }
+        if (c * 32 + 32 > ncols) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (c * 32 + j >= ncols) L[j] = -CUDART_INF_F;
+        }
+        float mx[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) mx[j] = fmaxf(L[j], L[j + 16]);
+#pragma unroll
+        for (int w = 8; w >= 1; w /= 2)
+#pragma unroll
+          for (int j = 0; j < w; ++j) mx[j] = fmaxf(mx[j], mx[j + w]);
+        const float mn = fmaxf(m, mx[0] * kLog2e);
+        if (mn == -CUDART_INF_F) return;  // nothing in range yet
+        float a4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < 32; ++j) a4[j & 3] += ex2_approx(fmaf(L[j], kLog2e, -mn));
+        const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+        s = (m == -CUDART_INF_F) ? acc : fmaf(s, ex2_approx(m - mn), acc);
+        m = mn;
+      };
+      constexpr int kChunks = BN / 2 / 32;
+      uint32_t buf[2][32];
+      tmem_ld_x32(ta, buf[0]);
+      tmem_ld_wait(buf[0]);
+#pragma unroll 1
+      for (int c = 0; c < kChunks; c += 2) {
+        tmem_ld_x32(ta + (c + 1) * 32, buf[1]);
+        chunk(c, buf[0]);
+        tmem_ld_wait(buf[1]);
+        if (c + 2 < kChunks)
+          tmem_ld_x32(ta + (c + 2) * 32, buf[0]);
+        else
+          release_tmem(tempty, lane);  // every column of this half is in registers
+        chunk(c + 1, buf[1]);
+        if (c + 2 < kChunks) tmem_ld_wait(buf[0]);
+      }
     }
+    if (row_ok && y_local >= 0) p.label_logit[row] = ly;
+    // the quadrant's second warp hands (m, s) to the first
+    uint64_t* bars = reinterpret_cast<uint64_t*>(part == 0 ? stg : stg - 4 * kStagingPerWarp);
+    float* x = reinterpret_cast<float*>(part == 1 ? stg : stg + 4 * kStagingPerWarp) + slot * 64;
+    const uint32_t full = smem_u32(&bars[slot]), empty = smem_u32(&bars[2 + slot]);
+    if (part == 1) {
+      if (use > 0 && !__all_sync(0xffffffffu, mbar_wait(empty, (use - 1) & 1u, abort, timeout_ns)))
+        return false;
+      x[lane] = m;
+      x[32 + lane] = s;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(full);
+      return true;
+    }
+    if (!__all_sync(0xffffffffu, mbar_wait(full, use & 1u, abort, timeout_ns))) return false;
+    const float m1 = x[lane], s1 = x[32 + lane];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty);
     if (row_ok) {
-      const size_t idx = static_cast<size_t>(nb) * p.N + row;
+      if (m1 != -CUDART_INF_F) {  // the second half has columns in range
+        const float mm = fmaxf(m, m1);
+        s = s * ex2_approx(m - mm) + s1 * ex2_approx(m1 - mm);
+        m = mm;
+      }
+      const size_t idx = static_cast<size_t>(col0 / BN) * p.N + row;
       p.part_m[idx] = m;
       p.part_s[idx] = s;
-      if (y_local >= 0) p.label_logit[row] = ly;
     }
+    return true;
   }
 };
 
@@ -282,6 +371,9 @@ struct FwdStatsEpi {
 // term of dHidden and dWeight exact.
 template <bool kSoftcap>
 struct DzEpi {
+  static constexpr int kEpiWarps = 4;
+  static constexpr int kStagingPerWarp = flce::kStagingPerWarp;
+  __device__ static void init_smem(uint8_t*) {}
   struct Params {
     const int64_t* labels;
     const float* lse;
@@ -307,16 +399,17 @@ struct DzEpi {
     return Pre{p.labels[p.t0 + row_l], p.lse[p.t0 + row_l]};
   }
 
-  __device__ static void tile(const Params& p, const Pre& pre, int m_base, int col0,
-                              uint32_t taddr, int q, int lane, uint8_t* stg,
-                              const CUtensorMap* out, uint32_t tempty, int& nstore, bool) {
+  __device__ static bool tile(const Params& p, const Pre& pre, int m_base, int col0,
+                              uint32_t taddr, int q, int lane, int, uint8_t* stg,
+                              const CUtensorMap* out, uint32_t tempty, int& nstore, bool,
+                              const volatile int*, unsigned long long) {
     // 64-column chunks whose store box starts inside the block (warp-uniform)
     const int y0 = m_base + q * 32;
     const int rem = p.cols - col0;
     const int nch = (y0 >= p.rows || rem <= 0) ? 0 : min(BN / 64, (rem + 63) / 64);
     if (nch == 0) {
       release_tmem(tempty, lane);
-      return;
+      return true;
     }
     const int row_l = y0 + lane;
     bool valid = false;
@@ -406,6 +499,7 @@ struct DzEpi {
       sub(sc + 1, buf[1], std::integral_constant<int, 1>{});
       if (sc + 2 < BN / 32) tmem_ld_wait(buf[0]);
     }
+    return true;
   }
 };
 
@@ -414,6 +508,9 @@ struct DzEpi {
 // when `reduce` (accumulation across chunks of the split reduction dimension).
 // g = grad_output * grad_scale, divided by max(n, 1) for 'mean'.
 struct StoreEpi {
+  static constexpr int kEpiWarps = 4;
+  static constexpr int kStagingPerWarp = flce::kStagingPerWarp;
+  __device__ static void init_smem(uint8_t*) {}
   struct Params {
     int out_row0;
     int reduce;
@@ -440,17 +537,17 @@ struct StoreEpi {
   };
   __device__ static Pre prepare(const Params& p, int, int, int) { return Pre{grad_factor(p)}; }
 
-  __device__ static void tile(const Params& p, const Pre& pre, int m_base, int col0,
-                              uint32_t taddr, int q, int lane, uint8_t* stg,
+  __device__ static bool tile(const Params& p, const Pre& pre, int m_base, int col0,
+                              uint32_t taddr, int q, int lane, int, uint8_t* stg,
                               const CUtensorMap* out, uint32_t tempty, int& nstore,
-                              bool empty) {
+                              bool empty, const volatile int*, unsigned long long) {
     const int y = p.out_row0 + m_base + q * 32;
     // 32-column chunks whose store box starts inside the output (warp-uniform)
     const int rem = p.x_limit - col0;
     const int nch = (y >= p.y_limit || rem <= 0) ? 0 : min(BN / 32, (rem + 31) / 32);
     if (nch == 0) {
       release_tmem(tempty, lane);
-      return;
+      return true;
     }
     // An empty K range contributes zeros: the accumulator was never written, so
     // its stale contents are not read (0 * stale could be NaN).
@@ -480,6 +577,7 @@ struct StoreEpi {
       }
       ++nstore;
     }
+    return true;
   }
 };
 
@@ -520,7 +618,7 @@ __device__ __forceinline__ void load_mn(uint32_t dst, const CUtensorMap* map, ui
 // last wave of one is filled by the other).  Operand majors are per problem.
 template <class Epi, int kCG, int kBN, bool kAMn0, bool kBMn0, bool kAMn1 = false,
           bool kBMn1 = false>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                    const __grid_constant__ CUtensorMap tmOut0, const __grid_constant__ CUtensorMap tmA1,
                    const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmOut1,
@@ -559,16 +657,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&bar_tfull[a]), 1);
-      mbar_init(smem_u32(&bar_tempty[a]), kEpiWarps * kCG);
+      mbar_init(smem_u32(&bar_tempty[a]), Epi::kEpiWarps * kCG);
     }
     mbar_init(smem_u32(&bar_drain), 1);
-    // each tile index is read by: the MMA issuer and 4 epilogue warps of the
-    // leader, and the producer and 4 epilogue warps of the peer
+    // each tile index is read by: the MMA issuer and the epilogue warps of
+    // the leader, and the producer and the epilogue warps of the peer
     for (int r = 0; r < kRing; ++r) {
       mbar_init(smem_u32(&ring_full[r]), 1);
-      mbar_init(smem_u32(&ring_empty[r]), (1 + kEpiWarps) * kCG);
+      mbar_init(smem_u32(&ring_empty[r]), (1 + Epi::kEpiWarps) * kCG);
     }
     abort_sh = 0;
+    Epi::init_smem(smem + kStages * Cfg::kStageBytes);
     fence_mbar_init();
     prefetch_tmap(&tmA0);
     prefetch_tmap(&tmB0);
@@ -893,8 +992,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- epilogue warps (they may read what the previous kernel
     // wrote, so they wait for it in either of the first two modes)
     if (g0.dep_wait == kDepBeforeLoads || g0.dep_wait == kDepBeforeStores) griddep_wait();
-    const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    uint8_t* stg = smem + kStages * Cfg::kStageBytes + (warp - 2) * kStagingPerWarp;
+    const int q = warp & 3;             // TMEM lane quadrant this warp may access
+    const int part = (warp - 2) >> 2;   // with 8 epilogue warps: which half of a bank
+    uint8_t* stg = smem + kStages * Cfg::kStageBytes + (warp - 2) * Epi::kStagingPerWarp;
     int it = 0;
     int nstore = 0;  // TMA stores issued by this warp (selects the staging buffer)
     bool ok = true;
@@ -946,9 +1046,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t taddr = tmem_base + bank * BN + (static_cast<uint32_t>(q * 32) << 16);
         const uint32_t tempty_local = smem_u32(&bar_tempty[bank]);
         const uint32_t tempty = (kCG == 1) ? tempty_local : mapa_shared(tempty_local, 0);
-        Epi::tile(prob ? ep1 : ep0, pre, m_base, nb * kBN + h * BN, taddr, q, lane, stg,
-                  prob ? &tmOut1 : &tmOut0, tempty, nstore, ga.k_blocks == 0);
+        if (!Epi::tile(prob ? ep1 : ep0, pre, m_base, nb * kBN + h * BN, taddr, q, lane, part,
+                       stg, prob ? &tmOut1 : &tmOut0, tempty, nstore, ga.k_blocks == 0,
+                       abort_flag, g0.timeout_ns)) {
+          ok = false;
+          break;
+        }
       }
+      if (!ok) break;
     }
     if (lane == 0) {
       bulk_wait_group_all();
