@@ -113,7 +113,8 @@ typedef enum flce_option {
   FLCE_OPT_WAIT_TIMEOUT_MS = 6, /* [1000] limit of every bounded wait inside a kernel (10 .. 60000) */
   FLCE_OPT_GRAD_TILE_N = 7,     /* [512] columns of a dHidden / dWeight tile: 512 or 256 (512 needs CTA pairs;
                                    with FLCE_OPT_CTA_GROUP = 1 tiles are 256 wide) */
-  FLCE_OPT_DZ_TILE_N = 8,       /* [256] columns of a backward dZ tile: 256 or 512 (as above) */
+  FLCE_OPT_DZ_TILE_N = 8,       /* [0] columns of a backward dZ tile: 256 or 512 (as above); 0: 512
+                                   without softcap, 256 with softcap */
   FLCE_OPT_FWD_TILE_N = 9,      /* [512] columns of a forward tile: 512 or 256 (as above) */
   FLCE_OPT_FWD_GROUP_M = 10,    /* [16] row tiles per raster group of the forward GEMM (1 .. 64): the
                                    group's hidden rows stay in L2 while the weight streams past */

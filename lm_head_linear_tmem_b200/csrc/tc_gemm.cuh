@@ -1,14 +1,16 @@
 // Persistent tcgen05 GEMM for the fused linear cross-entropy (FLCE).
 //
-// One CTA per SM (192 or 320 threads, up to ~225 KB shared memory, all 512
-// TMEM columns).  Warp roles:
+// One CTA per SM (320 threads, up to ~225 KB shared memory, all 512 TMEM
+// columns).  Warp roles:
 //   warp 0  TMA producer   (one thread): K-blocks of A and B into a stage ring
 //   warp 1  MMA issuer     (one thread): tcgen05.mma K=16 steps, fp32 in TMEM
-//   warps 2.. epilogue     4 or 8 warps (a trait of the epilogue), thread =
-//                          accumulator row: tcgen05.ld then an operation-
-//                          specific epilogue.  A warp may read only its TMEM
-//                          lane quadrant (warp % 4); with 8 warps two share a
-//                          quadrant and each takes half of a bank's columns.
+//   warps 2-9 epilogue     (a count the epilogue type sets), thread =
+//                          accumulator row.  A warp may read only its TMEM lane
+//                          quadrant (warp % 4), so two warps share a quadrant
+//                          and each takes half of a bank's columns: it loads
+//                          its 128 columns into registers, hands the TMEM bank
+//                          back at once (the next tile's MMAs wait for it), and
+//                          then runs the operation-specific epilogue.
 // Tile shapes (template parameters kCG, the CTA group, and kBN, the columns of
 // a tile):
 //   kCG = 1, kBN = 256  one CTA computes a 128 x 256 tile
@@ -58,7 +60,6 @@ constexpr int BN = 256;  // accumulator columns
 constexpr int BK = 64;
 constexpr int kABytes = BM * BK * 2;  // 16 KB
 constexpr int kStagingBuf = 4096;                 // 32 rows x 128 bytes
-constexpr int kStagingPerWarp = 2 * kStagingBuf;  // double buffered (TMA-store epilogues)
 constexpr uint32_t kTmemCols = 512;
 
 template <int kCG, int kBN = 256>
@@ -170,6 +171,19 @@ __device__ __forceinline__ void stage_row_128b(uint8_t* buf, int lane, const uin
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     uint4 v = make_uint4(w[4 * j + 0], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+    *reinterpret_cast<uint4*>(row + ((j ^ (lane & 7)) << 4)) = v;
+  }
+}
+
+// The same row from two halves: words 0-15 of `lo`, then words 0-15 of `hi`.
+__device__ __forceinline__ void stage_row_128b(uint8_t* buf, int lane, const uint32_t (&lo)[32],
+                                               const uint32_t (&hi)[32]) {
+  uint8_t* row = buf + lane * 128;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t(&w)[32] = j < 4 ? lo : hi;
+    const int b = 4 * (j & 3);
+    uint4 v = make_uint4(w[b + 0], w[b + 1], w[b + 2], w[b + 3]);
     *reinterpret_cast<uint4*>(row + ((j ^ (lane & 7)) << 4)) = v;
   }
 }
@@ -371,8 +385,10 @@ struct FwdStatsEpi {
 // term of dHidden and dWeight exact.
 template <bool kSoftcap>
 struct DzEpi {
-  static constexpr int kEpiWarps = 4;
-  static constexpr int kStagingPerWarp = flce::kStagingPerWarp;
+  // Eight warps: the two warps of a TMEM lane quadrant each take 128 of a
+  // bank's columns.  One 4 KiB staging buffer per warp (32 rows x 64 bf16).
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kStagingPerWarp = kStagingBuf;
   __device__ static void init_smem(uint8_t*) {}
   struct Params {
     const int64_t* labels;
@@ -400,13 +416,15 @@ struct DzEpi {
   }
 
   __device__ static bool tile(const Params& p, const Pre& pre, int m_base, int col0,
-                              uint32_t taddr, int q, int lane, int, uint8_t* stg,
+                              uint32_t taddr, int q, int lane, int part, uint8_t* stg,
                               const CUtensorMap* out, uint32_t tempty, int& nstore, bool,
                               const volatile int*, unsigned long long) {
-    // 64-column chunks whose store box starts inside the block (warp-uniform)
+    // this warp's columns: [h0, h0 + 128) of the block; 64-column stores whose
+    // box starts inside the block (warp-uniform)
+    const int h0 = col0 + part * (BN / 2);
     const int y0 = m_base + q * 32;
-    const int rem = p.cols - col0;
-    const int nch = (y0 >= p.rows || rem <= 0) ? 0 : min(BN / 64, (rem + 63) / 64);
+    const int rem = p.cols - h0;
+    const int nch = (y0 >= p.rows || rem <= 0) ? 0 : min(BN / 2 / 64, (rem + 63) / 64);
     if (nch == 0) {
       release_tmem(tempty, lane);
       return true;
@@ -418,86 +436,118 @@ struct DzEpi {
     if (row_l < p.rows) {
       const int64_t y = pre.y;
       valid = (y != p.ignore_index) && y >= 0 && y < p.v_total;
-      const int64_t c0 = static_cast<int64_t>(p.v0) + col0;
-      if (valid && y >= c0 && y < c0 + BN) y_local = static_cast<int>(y - c0);
+      const int64_t c0 = static_cast<int64_t>(p.v0) + h0;
+      if (valid && y >= c0 && y < c0 + BN / 2) y_local = static_cast<int>(y - c0);
       lse2 = pre.lse * kLog2e;
     }
     const uint32_t stg_u32 = smem_u32(stg);
-    // warp-uniform: does any row's label fall in this bank?
+    // warp-uniform: does any row's label fall in these columns?
     const bool any_label = __any_sync(0xffffffffu, y_local >= 0);
-    // 32-column sub-chunks, the next one's TMEM load in flight while this one
-    // is computed; every 64 columns are staged and stored
-    uint32_t packed[32];
-    // sub-chunk sc (32 columns) into half kH of `packed`; the odd half stages
-    // and stores the 64 columns
-    auto sub = [&](int sc, const uint32_t(&r)[32], auto half) {
-      constexpr int kH = decltype(half)::value;
-      if (sc >= 2 * nch) return;
-      float d[32], f[32];
+    // dZ/g of 32 columns (local columns c0l..c0l+31 of this warp), packed as
+    // 16 bf16 pairs into r[0..15] (in place: no second register array)
+    auto dz32 = [&](int c0l, uint32_t(&r)[32]) {
+      // d overwrites the logit it comes from
+      if constexpr (kSoftcap) {
+        float f[32];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float z = __uint_as_float(r[j]);
-        const float L = kSoftcap ? p.softcap * tanhf(z * p.inv_softcap) : z;
-        d[j] = ex2_approx(fmaf(L, kLog2e, -lse2));
-        if (kSoftcap) {
+        for (int j = 0; j < 32; ++j) {
+          const float L = p.softcap * tanhf(__uint_as_float(r[j]) * p.inv_softcap);
           const float u = L * p.inv_softcap;
           f[j] = fmaf(-u, u, 1.0f);
+          r[j] = __float_as_uint(ex2_approx(fmaf(L, kLog2e, -lse2)));
         }
-      }
-      if (any_label) {
+        if (any_label) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (c0l + j == y_local) r[j] = __float_as_uint(__uint_as_float(r[j]) - 1.0f);
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * f[j]);
+      } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          if (sc * 32 + j == y_local) d[j] -= 1.0f;
-      }
-      if (kSoftcap) {
+          r[j] = __float_as_uint(ex2_approx(fmaf(__uint_as_float(r[j]), kLog2e, -lse2)));
+        if (any_label) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) d[j] *= f[j];
+          for (int j = 0; j < 32; ++j)
+            if (c0l + j == y_local) r[j] = __float_as_uint(__uint_as_float(r[j]) - 1.0f);
+        }
       }
       if (any_label && p.resid != nullptr) {
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          if (sc * 32 + j == y_local)
-            p.resid[p.t0 + row_l] = d[j] - __bfloat162float(__float2bfloat16_rn(d[j]));
+          if (c0l + j == y_local) {
+            const float d = __uint_as_float(r[j]);
+            p.resid[p.t0 + row_l] = d - __bfloat162float(__float2bfloat16_rn(d));
+          }
       }
+      // pairs (2j, 2j+1) -> word j; word j is written after words 2j, 2j+1
+      // (>= j) are read
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        __nv_bfloat162 b2 =
-            __floats2bfloat162_rn(valid ? d[2 * j] : 0.0f, valid ? d[2 * j + 1] : 0.0f);
-        packed[kH * 16 + j] = *reinterpret_cast<uint32_t*>(&b2);
-      }
-      if (kH == 1) {
-        // Buffer = parity of this warp's store count: the store that last
-        // read this buffer is the one before the most recent, which
-        // wait_read<1> has retired.
-        const int b = nstore & 1;
-        if (lane == 0) bulk_wait_group_read<1>();
-        __syncwarp();
-        stage_row_128b(stg + b * kStagingBuf, lane, packed);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(out, stg_u32 + b * kStagingBuf, col0 + (sc >> 1) * 64, y0);
-          bulk_commit_group();
-        }
-        ++nstore;
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(valid ? __uint_as_float(r[2 * j]) : 0.0f,
+                                                  valid ? __uint_as_float(r[2 * j + 1]) : 0.0f);
+        r[j] = *reinterpret_cast<uint32_t*>(&b2);
       }
     };
-    // sub-chunks in pairs (one 64-column store each), the next one's TMEM load
-    // in flight while one is computed; the softcapped body stays rolled
-    uint32_t buf[2][32];
-    tmem_ld_x32(taddr, buf[0]);
-    tmem_ld_wait(buf[0]);
-#pragma unroll(kSoftcap ? 1 : BN / 64)
-    for (int sc = 0; sc < BN / 32; sc += 2) {
-      tmem_ld_x32(taddr + (sc + 1) * 32, buf[1]);
-      sub(sc, buf[0], std::integral_constant<int, 0>{});
-      tmem_ld_wait(buf[1]);
-      if (sc + 2 < BN / 32)
-        tmem_ld_x32(taddr + (sc + 2) * 32, buf[0]);
-      else
-        release_tmem(tempty, lane);  // every column of the bank is in registers
-      sub(sc + 1, buf[1], std::integral_constant<int, 1>{});
-      if (sc + 2 < BN / 32) tmem_ld_wait(buf[0]);
+    // 64 packed columns (local store index sidx) -> staging -> TMA store; the
+    // buffer is reused once the previous store has read it
+    auto store64 = [&](int sidx, const uint32_t(&lo)[32], const uint32_t(&hi)[32]) {
+      if (lane == 0) bulk_wait_group_read<0>();
+      __syncwarp();
+      stage_row_128b(stg, lane, lo, hi);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(out, stg_u32, h0 + sidx * 64, y0);
+        bulk_commit_group();
+      }
+      ++nstore;
+    };
+    if constexpr (!kSoftcap) {
+      // all 128 columns into registers, the TMEM half released at once
+      uint32_t r[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_x32(taddr + part * (BN / 2) + c * 32, r[c]);
+      tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) reg_fence(r[c]);
+      release_tmem(tempty, lane);
+#pragma unroll
+      for (int sidx = 0; sidx < 2; ++sidx) {
+        if (sidx < nch) {
+          dz32(sidx * 64, r[2 * sidx]);
+          dz32(sidx * 64 + 32, r[2 * sidx + 1]);
+          store64(sidx, r[2 * sidx], r[2 * sidx + 1]);
+        }
+      }
+    } else {
+      // softcapped: 32-column sub-chunks, the next one's TMEM load in flight;
+      // the tanh body is kept rolled to bound code size
+      const uint32_t ta = taddr + part * (BN / 2);
+      uint32_t buf[2][32];
+      tmem_ld_x32(ta, buf[0]);
+      tmem_ld_wait(buf[0]);
+#pragma unroll 1
+      for (int sidx = 0; sidx < 2; ++sidx) {
+        uint32_t lo[32];
+        tmem_ld_x32(ta + (2 * sidx + 1) * 32, buf[1]);
+        if (sidx < nch) {
+          dz32(sidx * 64, buf[0]);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) lo[j] = buf[0][j];
+        }
+        tmem_ld_wait(buf[1]);
+        if (sidx == 0)
+          tmem_ld_x32(ta + 64, buf[0]);
+        else
+          release_tmem(tempty, lane);  // every column of this half is in registers
+        if (sidx < nch) {
+          dz32(sidx * 64 + 32, buf[1]);
+          store64(sidx, lo, buf[1]);
+        }
+        if (sidx == 0) tmem_ld_wait(buf[0]);
+      }
     }
     return true;
   }
@@ -508,8 +558,10 @@ struct DzEpi {
 // when `reduce` (accumulation across chunks of the split reduction dimension).
 // g = grad_output * grad_scale, divided by max(n, 1) for 'mean'.
 struct StoreEpi {
-  static constexpr int kEpiWarps = 4;
-  static constexpr int kStagingPerWarp = flce::kStagingPerWarp;
+  // Eight warps: the two warps of a TMEM lane quadrant each take 128 of a
+  // bank's columns.  One 4 KiB staging buffer per warp (32 rows x 32 fp32).
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kStagingPerWarp = kStagingBuf;
   __device__ static void init_smem(uint8_t*) {}
   struct Params {
     int out_row0;
@@ -538,13 +590,15 @@ struct StoreEpi {
   __device__ static Pre prepare(const Params& p, int, int, int) { return Pre{grad_factor(p)}; }
 
   __device__ static bool tile(const Params& p, const Pre& pre, int m_base, int col0,
-                              uint32_t taddr, int q, int lane, int, uint8_t* stg,
+                              uint32_t taddr, int q, int lane, int part, uint8_t* stg,
                               const CUtensorMap* out, uint32_t tempty, int& nstore,
                               bool empty, const volatile int*, unsigned long long) {
+    // this warp's columns: [h0, h0 + 128); 32-column stores whose box starts
+    // inside the output (warp-uniform)
+    const int h0 = col0 + part * (BN / 2);
     const int y = p.out_row0 + m_base + q * 32;
-    // 32-column chunks whose store box starts inside the output (warp-uniform)
-    const int rem = p.x_limit - col0;
-    const int nch = (y >= p.y_limit || rem <= 0) ? 0 : min(BN / 32, (rem + 31) / 32);
+    const int rem = p.x_limit - h0;
+    const int nch = (y >= p.y_limit || rem <= 0) ? 0 : min(BN / 2 / 32, (rem + 31) / 32);
     if (nch == 0) {
       release_tmem(tempty, lane);
       return true;
@@ -553,29 +607,36 @@ struct StoreEpi {
     // its stale contents are not read (0 * stale could be NaN).
     const float g = empty ? 0.0f : pre.g;
     const uint32_t stg_u32 = smem_u32(stg);
-#pragma unroll 1
-    for (int c = 0; c < nch; ++c) {
-      uint32_t r[32];
-      tmem_ld_x32(taddr + c * 32, r);
-      tmem_ld_wait();
-      if (c == nch - 1) release_tmem(tempty, lane);
+    // all 128 columns into registers, the TMEM half released at once
+    uint32_t r[4][32];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) r[j] = empty ? 0u : __float_as_uint(__uint_as_float(r[j]) * g);
-      const int b = nstore & 1;  // see DzEpi
-      if (lane == 0) bulk_wait_group_read<1>();
-      __syncwarp();
-      stage_row_128b(stg + b * kStagingBuf, lane, r);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        const int x = col0 + c * 32;
-        if (p.reduce)
-          tma_reduce_add_2d(out, stg_u32 + b * kStagingBuf, x, y);
-        else
-          tma_store_2d(out, stg_u32 + b * kStagingBuf, x, y);
-        bulk_commit_group();
+    for (int c = 0; c < 4; ++c) tmem_ld_x32(taddr + part * (BN / 2) + c * 32, r[c]);
+    tmem_ld_wait();
+#pragma unroll
+    for (int c = 0; c < 4; ++c) reg_fence(r[c]);
+    release_tmem(tempty, lane);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (c < nch) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          r[c][j] = empty ? 0u : __float_as_uint(__uint_as_float(r[c][j]) * g);
+        // the buffer is reused once the previous store has read it
+        if (lane == 0) bulk_wait_group_read<0>();
+        __syncwarp();
+        stage_row_128b(stg, lane, r[c]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int x = h0 + c * 32;
+          if (p.reduce)
+            tma_reduce_add_2d(out, stg_u32, x, y);
+          else
+            tma_store_2d(out, stg_u32, x, y);
+          bulk_commit_group();
+        }
+        ++nstore;
       }
-      ++nstore;
     }
     return true;
   }

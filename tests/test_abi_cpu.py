@@ -127,7 +127,7 @@ def test_options_host_side(lib):
     v = ctypes.c_int64()
     defaults = {"cta_group": 2, "bwd_compact": 1, "bwd_fuse": 1, "mn3d": 1,
                 "chunk_tokens": 16384, "chunk_vocab": 16384, "wait_timeout_ms": 1000,
-                "grad_tile_n": 512, "dz_tile_n": 256, "fwd_tile_n": 512, "fwd_group_m": 16,
+                "grad_tile_n": 512, "dz_tile_n": 0, "fwd_tile_n": 512, "fwd_group_m": 16,
                 "dz_group_m": 16, "grad_group_m": 8, "fwd_dynamic": 1,
                 "dz_buffers": 1, "fwd_compact": 1}
     assert set(defaults) == set(_native.OPTIONS)
@@ -137,6 +137,7 @@ def test_options_host_side(lib):
     for name, bad in (("cta_group", 3), ("cta_group", 0), ("bwd_compact", 2),
                       ("chunk_tokens", 100), ("chunk_vocab", 1 << 21),
                       ("wait_timeout_ms", 5), ("grad_tile_n", 384), ("dz_tile_n", 128),
+                      ("grad_tile_n", 0), ("fwd_tile_n", 0),
                       ("fwd_tile_n", 1024), ("fwd_group_m", 0), ("grad_group_m", 65)):
         assert lib.flce_set_option(_native.OPTIONS[name], bad) == ARG, (name, bad)
         assert _native.get_option(name) == defaults[name]

@@ -386,7 +386,8 @@ def test_degenerate_shapes(N, H, V, dtype):
 
 
 @pytest.mark.parametrize("switch", ["cta_group=1", "bwd_fuse=0", "bwd_compact=0", "mn3d=0",
-                                    "grad_tile_n=256", "dz_tile_n=512", "fwd_tile_n=256",
+                                    "grad_tile_n=256", "dz_tile_n=512", "dz_tile_n=256",
+                                    "fwd_tile_n=256",
                                     "fwd_dynamic=0", "dz_buffers=2", "dz_buffers=2,bwd_fuse=0",
                                     "dz_buffers=2,cta_group=1", "fwd_group_m=3,dz_group_m=2,"
                                     "grad_group_m=1", "fwd_compact=0", "fwd_compact=0,cta_group=1"])
@@ -394,7 +395,7 @@ def test_alternative_paths(switch):
     """Each schedule option of the library selects another correct path: single-CTA
     128 x 256 tiles, separate dHidden and dWeight launches, no row compaction (and
     so no exact label term), 2-D views for MN-major operands, 256-column gradient
-    and forward tiles, 512-column dZ tiles, round-robin forward tiles, two dZ
+    and forward tiles, either dZ tile width, round-robin forward tiles, two dZ
     blocks (9 chunks here, so a dZ launch waits on the gradient launches two
     chunks back before it overwrites their block), other raster groups, a
     forward over every row instead of the compacted ones."""
@@ -406,12 +407,14 @@ def test_alternative_paths(switch):
     compare(got, inp.hidden, inp.weight, inp.labels, 2.0, "mean", grad_scale=0.7)
 
 
+@pytest.mark.parametrize("softcap", [0.0, 3.0])
 @pytest.mark.parametrize("width", [256, 512])
 @pytest.mark.parametrize("shape", [(300, 200, 1000), (37, 8, 700), (700, 1000, 1300),
                                    (4500, 136, 9000)])
-def test_tile_widths(width, shape):
-    """Every tensor-core GEMM with 256- or 512-column tiles on ragged shapes: the
-    second 256-column bank of a 512-column tile may lie wholly past the vocabulary
+def test_tile_widths(width, shape, softcap):
+    """Every tensor-core GEMM with 256- or 512-column tiles on ragged shapes, with and
+    without softcap (each epilogue has a separate softcapped body): the second
+    256-column bank of a 512-column tile may lie wholly past the vocabulary
     (forward, dZ) or past H (dHidden, dWeight: H = 8, 136, 200, 1000), and the
     multi-chunk case crosses 5 x 5 backward chunks."""
     N, H, V = shape
@@ -419,8 +422,8 @@ def test_tile_widths(width, shape):
     chunked = G.chunks(*SMALL_CHUNKS) if N > 4000 else contextlib.nullcontext()
     with _native.options(fwd_tile_n=width, dz_tile_n=width, grad_tile_n=width), chunked:
         got = run(G.bf16_tensor(inp.hidden_bits), G.bf16_tensor(inp.weight_bits),
-                  G.labels_tensor(inp.labels), 3.0, "sum", grad_scale=0.5)
-    compare(got, inp.hidden, inp.weight, inp.labels, 3.0, "sum", grad_scale=0.5)
+                  G.labels_tensor(inp.labels), softcap, "sum", grad_scale=0.5)
+    compare(got, inp.hidden, inp.weight, inp.labels, softcap, "sum", grad_scale=0.5)
 
 
 @pytest.mark.parametrize("softcap", [0.05, 1.0])
