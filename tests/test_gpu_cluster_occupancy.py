@@ -14,8 +14,8 @@ import torch
 
 pytestmark = pytest.mark.gpu
 
-THREADS = 192          # threads of a GEMM CTA (producer, MMA and 4 epilogue warps)
-SMEM = 230400          # dynamic shared memory of a GEMM CTA (operand ring + staging)
+THREADS = 320          # threads of a GEMM CTA (producer, MMA and 8 epilogue warps)
+SMEM = 230400          # dynamic shared memory of the largest GEMM CTA (ring + staging)
 SOURCE = (b'extern "C" __global__ void occupancy_probe(int* p) {'
           b' extern __shared__ int s[]; if (p) p[threadIdx.x] = s[threadIdx.x]; }')
 
