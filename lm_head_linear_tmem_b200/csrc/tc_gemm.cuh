@@ -94,6 +94,17 @@ constexpr uint32_t kStatusLabelRange = 1u;
 constexpr uint32_t kStatusTimeout = 2u;
 
 constexpr float kLog2e = 1.4426950408889634f;
+
+// tanh from one SFU exp2 and one fast division, by the identity
+// tanh(x) = sign(x) * (1 - e^{-2|x|}) / (1 + e^{-2|x|}).  e^{-2|x|} lies in
+// (0, 1] with relative (so also absolute) error about 2^-22, and the division
+// by a value in [1, 2] adds about as much: the absolute error of the result
+// stays near 2^-21 for every x, which the softcap s scales to s * 2^-21 in the
+// capped logit (1.4e-5 at s = 30).
+__device__ __forceinline__ float tanh_exp2(float x) {
+  const float e = ex2_approx(-2.0f * kLog2e * fabsf(x));
+  return copysignf(__fdividef(1.0f - e, 1.0f + e), x);
+}
 constexpr float kLn2 = 0.6931471805599453f;
 
 struct GemmArgs {
@@ -295,7 +306,8 @@ struct FwdStatsEpi {
       auto chunk = [&](int c, const uint32_t(&r)[32]) {
         float L[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) L[j] = p.softcap * tanhf(__uint_as_float(r[j]) * p.inv_softcap);
+        for (int j = 0; j < 32; ++j)
+          L[j] = p.softcap * tanh_exp2(__uint_as_float(r[j]) * p.inv_softcap);
         if (any_label) {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
@@ -451,7 +463,7 @@ struct DzEpi {
         float f[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float L = p.softcap * tanhf(__uint_as_float(r[j]) * p.inv_softcap);
+          const float L = p.softcap * tanh_exp2(__uint_as_float(r[j]) * p.inv_softcap);
           const float u = L * p.inv_softcap;
           f[j] = fmaf(-u, u, 1.0f);
           r[j] = __float_as_uint(ex2_approx(fmaf(L, kLog2e, -lse2)));
@@ -686,6 +698,7 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
                    const GemmArgs g0, const GemmArgs g1, const typename Epi::Params ep0,
                    const typename Epi::Params ep1) {
   using Cfg = TileCfg<kCG, kBN>;
+  static_assert(Epi::kEpiWarps == 8, "two epilogue warps per TMEM lane quadrant, half a bank each");
   constexpr int kStages = Cfg::kStages;
   constexpr int kBanks = Cfg::kBanks;
   // K-blocks of a 512-column tile issued on bank 0 alone while bank 1 still
@@ -1054,7 +1067,7 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 1)
     // wrote, so they wait for it in either of the first two modes)
     if (g0.dep_wait == kDepBeforeLoads || g0.dep_wait == kDepBeforeStores) griddep_wait();
     const int q = warp & 3;             // TMEM lane quadrant this warp may access
-    const int part = (warp - 2) >> 2;   // with 8 epilogue warps: which half of a bank
+    const int part = (warp - 2) >> 2;   // which half of a bank
     uint8_t* stg = smem + kStages * Cfg::kStageBytes + (warp - 2) * Epi::kStagingPerWarp;
     int it = 0;
     int nstore = 0;  // TMA stores issued by this warp (selects the staging buffer)
