@@ -11,7 +11,7 @@
 namespace flce {
 
 constexpr int kMergeRows = 32;
-constexpr int kMergeSplit = 8;
+constexpr int kMergeSplit = 32;
 constexpr int kLossThreads = 256;
 constexpr int kFinalThreads = 1024;
 
@@ -29,7 +29,7 @@ __device__ __forceinline__ void merge_ms(float& M, float& S, float m, float s) {
 
 // lse = ln 2 * (M + log2 S) over all vocab tiles of a row, for the rows that
 // take part in the loss; a row whose label is ignore_index (or outside
-// [0, V)) gets lse 0 and no merge.  Block (32 rows, 8 splits); grid ceil(N/32).
+// [0, V)) gets lse 0 and no merge.  Block (32 rows, 32 splits); grid ceil(N/32).
 //   perm == nullptr: the partials are indexed by row; a row's label decides.
 //   perm != nullptr: the forward ran on compacted rows: partial column j is
 //     compact row j, the original row perm[j]; the first *n_valid compact rows
@@ -424,14 +424,15 @@ constexpr int kFixSeg = 64;
 constexpr int kFixCols = 256;
 constexpr int kFixThreads = kFixCols / 2;
 
+// Each dWeight element receives at most one such addition (a label's rows form
+// one run), so a reduction without a returned value (no thread waits on the
+// old value) leaves the result as reproducible as a read-add-write.
 __device__ __forceinline__ void dw_fix_add(float* d_weight, int64_t v, int64_t V, int H, int col,
                                            float g, float a0, float a1) {
   if (v < 0 || v >= V) return;  // a label the forward reported as out of range
-  float2* o = reinterpret_cast<float2*>(d_weight + static_cast<size_t>(v) * H + col);
-  float2 cur = *o;
-  cur.x = fmaf(g, a0, cur.x);
-  cur.y = fmaf(g, a1, cur.y);
-  *o = cur;
+  float* o = d_weight + static_cast<size_t>(v) * H + col;
+  atomicAdd(o, g * a0);
+  atomicAdd(o + 1, g * a1);
 }
 
 __global__ void __launch_bounds__(kFixThreads)
